@@ -1,0 +1,58 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kvc.h"
+
+namespace kvc {
+
+// Geometry and pointers resolved once on the host for a call.
+struct CacheView {
+    const void *k_pool;
+    const void *v_pool;
+    int64_t num_pages;
+    int32_t page_size, head_dim, dtype, max_pages_per_row;
+    int32_t *block_table;
+    int32_t *row_len;
+    int32_t *slot_pos;
+    uint8_t *slot_label;
+    int32_t num_seqs, num_layers, num_kv_heads;
+    int32_t rows;
+    int64_t max_slots;
+};
+
+struct QueryView {
+    const void *q;
+    float *lse;
+    const int32_t *q_pos;
+    const int32_t *num_q;
+    int32_t max_q, num_q_heads, group;
+};
+
+// Each launcher enqueues its kernels on `stream` and returns cudaGetLastError().
+cudaError_t launch_score_simt(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
+                              int32_t *status, cudaStream_t stream);
+cudaError_t launch_lse_simt(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream);
+cudaError_t launch_score_tc(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
+                            int32_t *status, cudaStream_t stream, char *err, size_t errlen);
+cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, float decay, float hit_mass,
+                        bool binary, int32_t *status, cudaStream_t stream);
+cudaError_t launch_select(const CacheView &c, const float *crf, const int32_t *budget, uint32_t protect,
+                          uint8_t *keep, int32_t *kept, int32_t *status, cudaStream_t stream);
+cudaError_t launch_plan(const CacheView &c, const uint8_t *keep, const int32_t *kept, int32_t *move_src,
+                        int32_t *move_dst, int32_t *num_moves, int32_t *status, cudaStream_t stream);
+cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const int32_t *move_dst,
+                           const int32_t *num_moves, const int32_t *new_len, float *crf, int32_t *freed,
+                           int64_t freed_capacity, int64_t *num_freed, int64_t *row_offsets,
+                           int32_t *status, cudaStream_t stream);
+cudaError_t launch_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params &p,
+                                cudaStream_t stream);
+cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab, void *state,
+                           int32_t *budget, float *conf_out, const kvc_ratchet_params &p, int32_t *status,
+                           cudaStream_t stream);
+
+size_t ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params &p);
+
+}  // namespace kvc

@@ -1,0 +1,699 @@
+// Tensor-core scoring from the LSE (bf16 caches), sm_100a.
+//
+// "ActKV Dissected", Component 3: the softmax log-sum-exp is a byproduct of paged
+// attention, so each query's attention probabilities are recovered as its logits
+// minus the LSE, with no gather of the attention matrix and no recompute of the
+// attention itself; Component 1: an entry's score is the attention tallied over all
+// action tokens (here: over the query set and the query heads of the GQA group).
+//
+//   s[row][i] = sum_{j, g} [q_pos_j >= slot_pos_i] * 2^( (q_{j,g} . k_i) * log2(e)/sqrt(D)
+//                                                      - lse_{j,g} * log2(e) )
+//
+// Design (one persistent CTA per SM, 10 warps):
+//   warp 0     producer: per 256-key tile, 16 TMA page loads (one 16x64 bf16 box per
+//              page and 64-column half of D) gather the K tile from the paged pool into
+//              a 128B-swizzled A operand; per 128-column block of the query set, TMA
+//              loads of the Q block (4-D map: D, head, query, seq*layer) into a stage
+//              ring; per block it also publishes the columns' (lse*log2e, q_pos) and,
+//              once per tile, the keys' positions, through a metadata ring.
+//   warp 1     TMEM owner and MMA issuer: for each block, two M=128 x N=128 x K=D
+//              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) into one of two TMEM
+//              accumulator buffers (4 x 128 of the 512 columns).
+//   warps 2-9  epilogue: thread = key (TMEM lane); tcgen05.ld 32 columns at a time,
+//              x = acc * log2e/sqrt(D) - L_col, causal select, ex2, sum in registers.
+//              No cross-thread reduction; one coalesced store per key per tile.
+// Blocks whose queries all precede the tile's first key are skipped entirely
+// (no load, no MMA, no epilogue work).  Every barrier wait is bounded (about one
+// second of global time); on expiry the kernel records KVC_DEV_TIMEOUT, drains its
+// own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kvc {
+namespace {
+
+constexpr int kTileKeys = 256;          // keys per tile (two M=128 MMAs)
+constexpr int kPagesPerTile = 16;       // page_size 16
+constexpr int kCols = 128;              // MMA N: query columns per block
+constexpr int kMeta = 8;                // metadata ring depth
+constexpr int kMaxBlocks = 256;         // column blocks per sequence
+constexpr int kThreads = 320;           // 10 warps
+constexpr int kEpiWarps = 8;
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+struct alignas(16) Item {
+    float L[kCols];                     // lse * log2(e) per column (+inf for an absent column)
+    int32_t qp[kCols];                  // q_pos per column (INT32_MIN for an absent column)
+    int32_t kpos[kTileKeys];            // FIRST items: slot_pos of the tile's keys
+    uint32_t kvalid[8];                 // FIRST items: keys that are present and readable
+    int32_t cq_min[4], cq_max[4];       // per 32-column chunk: min/max q_pos of its valid columns
+    int32_t row, tile, blk, flags;      // blk < 0: tile with no visible block; row < 0: end of work
+    int32_t n_keys, valid_cols, pad0, pad1;
+};
+static_assert(sizeof(Item) % 16 == 0, "items hold float4-read arrays");
+constexpr int kFirst = 1, kLast = 2;
+
+struct Ctrl {
+    uint64_t q_full[8], q_empty[8];
+    uint64_t a_full, a_empty;
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t m_full[kMeta], m_empty[kMeta];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int32_t abort;
+    int32_t blk_qmin[kMaxBlocks], blk_qmax[kMaxBlocks];
+};
+
+struct TcArgs {
+    CacheView c;
+    QueryView q;
+    float *scores;
+    int32_t *status;
+    int accumulate;
+    int nqb;           // queries per column block (floor(128 / G))
+    int tiles_per_row;
+    int64_t total_tiles;
+    float scale_log2e; // log2(e) / sqrt(D)
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait; false when the CTA is aborting or the wait gave up (then the abort flag is set).
+__device__ bool mbar_wait(uint64_t *bar, uint32_t parity, Ctrl &ctl, int32_t *status, int row) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 63) == 0) {
+            if (*(volatile int32_t *)&ctl.abort) return false;
+            if (now_ns() - t0 > kTimeoutNs) {
+                report(status, KVC_DEV_TIMEOUT, row);
+                atomicExch(&ctl.abort, 1);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y, int z,
+                                            int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
+// 128B-swizzled K-major operand: 8-row groups 1024 bytes apart, version 1, layout SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
+           ((uint64_t)2 << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M = 128, N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kCols >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------- shared memory plan
+template <int D>
+struct Plan {
+    static constexpr int kChunks = D / 64;                       // 128-byte K chunks
+    static constexpr int kABytes = kTileKeys * D * 2;           // whole K tile
+    static constexpr int kBBytes = kCols * D * 2;                // one Q block
+    static constexpr int kStages = D == 128 ? 4 : 8;
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kABytes;
+    static constexpr int kOffItems = kOffB + kStages * kBBytes;
+    static constexpr int kOffCtrl = kOffItems + kMeta * (int)sizeof(Item);
+    static constexpr int kBytes = kOffCtrl + (int)sizeof(Ctrl) + 1024;  // + alignment slack
+};
+
+// ---------------------------------------------------------------- the kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q, TcArgs a) {
+    using PL = Plan<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem + PL::kOffA;
+    uint8_t *sB = smem + PL::kOffB;
+    Item *items = reinterpret_cast<Item *>(smem + PL::kOffItems);
+    Ctrl &ctl = *reinterpret_cast<Ctrl *>(smem + PL::kOffCtrl);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const CacheView &c = a.c;
+
+    // zero the operand buffers once so rows no load ever fills hold finite values
+    for (int i = threadIdx.x; i < (PL::kABytes + PL::kStages * PL::kBBytes) / 16; i += kThreads)
+        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PL::kStages; ++s) {
+            mbar_init(&ctl.q_full[s], 1);
+            mbar_init(&ctl.q_empty[s], 1);
+        }
+        mbar_init(&ctl.a_full, 1);
+        mbar_init(&ctl.a_empty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl.acc_full[b], 1);
+            mbar_init(&ctl.acc_empty[b], kEpiWarps);
+        }
+        for (int k = 0; k < kMeta; ++k) {
+            mbar_init(&ctl.m_full[k], 1);
+            mbar_init(&ctl.m_empty[k], 1 + kEpiWarps);
+        }
+        mbar_init(&ctl.drain, 1);
+        ctl.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl.tmem_base)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    const int G = a.q.group, Hq = a.q.num_q_heads, nqb = a.nqb;
+    const int RPS = c.num_layers * c.num_kv_heads;
+
+    if (warp == 0) {
+        // ============================== producer ==============================
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
+        uint32_t qs = 0, qph = 0, aph = 0, mk = 0, mph = 0;
+        int cur_seq = -1, nblk = 0, nq = 0;
+        const uint32_t a_tx_page = 16 * 128;                 // one 16-row, 128-byte box
+        const uint32_t q_tx = (uint32_t)(G * nqb) * 128u;    // one Q box per 64-column chunk
+        bool ok = true;
+        for (int64_t tid = blockIdx.x; ok && tid < a.total_tiles; tid += gridDim.x) {
+            const int64_t rr = tid % RPS, rest = tid / RPS;
+            const int t = (int)(rest % a.tiles_per_row), seq = (int)(rest / a.tiles_per_row);
+            const int row = seq * RPS + (int)rr;
+            const int n = c.row_len[row];
+            if (n < 0 || n > c.max_slots) {
+                if (t == 0 && lane == 0) report(a.status, KVC_DEV_BAD_LENGTH, row);
+                continue;
+            }
+            const int k0 = t * kTileKeys;
+            if (k0 >= n) continue;
+            const int n_keys = min(kTileKeys, n - k0);
+            const int layer = (int)(rr / c.num_kv_heads), kvh = (int)(rr % c.num_kv_heads);
+            if (seq != cur_seq) {
+                cur_seq = seq;
+                nq = min(a.q.num_q[seq], a.q.max_q);
+                nblk = (nq + nqb - 1) / nqb;
+                for (int b = lane; b < nblk; b += 32) {
+                    int mn = INT32_MAX, mx = INT32_MIN;
+                    const int j1 = min(nq, (b + 1) * nqb);
+                    for (int j = b * nqb; j < j1; ++j) {
+                        const int p = a.q.q_pos[(int64_t)seq * a.q.max_q + j];
+                        mn = min(mn, p);
+                        mx = max(mx, p);
+                    }
+                    ctl.blk_qmin[b] = mn;
+                    ctl.blk_qmax[b] = mx;
+                }
+                __syncwarp();
+            }
+            // pages of the tile (lanes 0..15) and keys' positions (8 per lane)
+            int page = -1;
+            bool page_ok = false;
+            if (lane < kPagesPerTile && k0 + lane * 16 < n) {
+                page = c.block_table[(int64_t)row * c.max_pages_per_row + t * kPagesPerTile + lane];
+                page_ok = page >= 0 && page < c.num_pages;
+                if (!page_ok) report(a.status, KVC_DEV_BAD_PAGE, row);
+            }
+            const unsigned okmask = __ballot_sync(0xffffffffu, page_ok);
+            int kp[8];
+            int kmin = INT32_MAX;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int key = i * 32 + lane;
+                const bool v = key < n_keys && ((okmask >> (key >> 4)) & 1u);
+                kp[i] = v ? c.slot_pos[(int64_t)row * c.max_slots + k0 + key] : INT32_MAX;
+                if (v) kmin = min(kmin, kp[i]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+            // visible blocks: some query at or after the tile's first key position
+            int first_vis = -1, last_vis = -1;
+            for (int b0 = 0; b0 < nblk; b0 += 32) {
+                const int b = b0 + lane;
+                const bool v = b < nblk && ctl.blk_qmax[b] >= kmin;
+                const unsigned m = __ballot_sync(0xffffffffu, v);
+                if (m) {
+                    if (first_vis < 0) first_vis = b0 + __ffs(m) - 1;
+                    last_vis = b0 + 31 - __clz(m);
+                }
+            }
+            auto fill_tile_part = [&](Item &it, int flags) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) it.kpos[i * 32 + lane] = kp[i];
+                if (lane < 8) {
+                    uint32_t w = 0;
+                    for (int bit = 0; bit < 32; ++bit) {
+                        const int key = lane * 32 + bit;
+                        if (key < n_keys && ((okmask >> (key >> 4)) & 1u)) w |= 1u << bit;
+                    }
+                    it.kvalid[lane] = w;
+                }
+                if (lane == 0) {
+                    it.row = row;
+                    it.tile = t;
+                    it.n_keys = n_keys;
+                    it.flags = flags;
+                }
+            };
+            if (first_vis < 0) {
+                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                Item &it = items[mk];
+                fill_tile_part(it, kFirst | kLast);
+                if (lane == 0) {
+                    it.blk = -1;
+                    it.valid_cols = 0;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
+                if (++mk == kMeta) { mk = 0; mph ^= 1; }
+                continue;
+            }
+            // K tile: one box per (page, 64-column chunk)
+            if (!mbar_wait(&ctl.a_empty, aph ^ 1, ctl, a.status, row)) { ok = false; break; }
+            aph ^= 1;
+            if (lane == 0) mbar_expect_tx(&ctl.a_full, (uint32_t)__popc(okmask) * a_tx_page * PL::kChunks);
+            __syncwarp();
+            if (page_ok) {
+                const int half = lane >> 3, r0 = (lane & 7) * 16;
+#pragma unroll
+                for (int kc = 0; kc < PL::kChunks; ++kc) {
+                    const uint32_t dst = smem_u32(sA + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
+                    tma_load_2d(dst, &tmap_k, &ctl.a_full, kc * 64, page * 16);
+                }
+            }
+            // column metadata of a block: 4 columns per lane, prefetched one block ahead
+            auto load_cols = [&](int b, float (&L)[4], int (&P)[4]) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = u * 32 + lane, jl = col / G, g = col % G, j = b * nqb + jl;
+                    L[u] = INFINITY;
+                    P[u] = INT32_MIN;
+                    if (jl < nqb && j < nq) {
+                        const float l = a.q.lse[((int64_t)(seq * c.num_layers + layer) * Hq + kvh * G + g) * a.q.max_q + j];
+                        if (l == -INFINITY) {
+                            // a column that saw no key contributes nothing
+                        } else if (!is_finite(l)) {
+                            report(a.status, KVC_DEV_NONFINITE, row);
+                        } else {
+                            L[u] = l * 1.4426950408889634f;
+                            P[u] = a.q.q_pos[(int64_t)seq * a.q.max_q + j];
+                        }
+                    }
+                }
+            };
+            float L[4], Ln[4];
+            int P[4], Pn[4];
+            load_cols(first_vis, L, P);
+            for (int b = first_vis; b >= 0;) {
+                int bn = -1;
+                for (int x = b + 1; x <= last_vis; ++x)
+                    if (ctl.blk_qmax[x] >= kmin) { bn = x; break; }
+                if (bn >= 0) load_cols(bn, Ln, Pn);
+                // Q block b
+                if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_expect_tx(&ctl.q_full[qs], q_tx * PL::kChunks);
+#pragma unroll
+                    for (int kc = 0; kc < PL::kChunks; ++kc) {
+                        const uint32_t dst = smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128));
+                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, kvh * G, b * nqb, seq * c.num_layers + layer);
+                    }
+                }
+                if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
+                // metadata item
+                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                Item &it = items[mk];
+                const int flags = (b == first_vis ? kFirst : 0) | (b == last_vis ? kLast : 0);
+                if (flags & kFirst) fill_tile_part(it, flags);
+                int vq = min(nqb, nq - b * nqb);
+                const int vcols = vq * G;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    it.L[u * 32 + lane] = L[u];
+                    it.qp[u * 32 + lane] = P[u];
+                    int mn = P[u] == INT32_MIN ? INT32_MAX : P[u], mx = P[u];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    }
+                    if (lane == 0) {
+                        it.cq_min[u] = mn;
+                        it.cq_max[u] = mx;
+                    }
+                }
+                if (lane == 0) {
+                    it.row = row;
+                    it.tile = t;
+                    it.blk = b;
+                    it.flags = flags;
+                    it.n_keys = n_keys;
+                    it.valid_cols = vcols;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
+                if (++mk == kMeta) { mk = 0; mph ^= 1; }
+                b = bn;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    L[u] = Ln[u];
+                    P[u] = Pn[u];
+                }
+            }
+        }
+        // end-of-work marker
+        if (ok && mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, -1)) {
+            if (lane == 0) {
+                items[mk].row = -1;
+                mbar_arrive(&ctl.m_full[mk]);
+            }
+        }
+        if (!ok || ctl.abort) {
+            // drain our own copies before the CTA can exit: every issued TMA phase completes
+            for (int s = 0; s < PL::kStages; ++s) {
+                const uint64_t t0 = now_ns();
+                while (!mbar_test(&ctl.q_full[s], (qph ^ (s < (int)qs ? 0u : 1u)) & 1u) && now_ns() - t0 < kTimeoutNs) {}
+            }
+            const uint64_t t0 = now_ns();
+            while (!mbar_test(&ctl.a_full, aph ^ 1) && now_ns() - t0 < kTimeoutNs) {}
+        }
+    } else if (warp == 1) {
+        // ============================== MMA issuer ==============================
+        uint32_t qs = 0, qph = 0, aph = 0, mk = 0, mph = 0, ab = 0, abph = 0;
+        bool issued = false;
+        for (;;) {
+            if (!mbar_wait(&ctl.m_full[mk], mph, ctl, a.status, -1)) break;
+            const Item &it = items[mk];
+            const int row = it.row;
+            if (row < 0) break;
+            const int blk = it.blk, flags = it.flags;
+            if (blk >= 0) {
+                if (flags & kFirst) {
+                    if (!mbar_wait(&ctl.a_full, aph, ctl, a.status, row)) break;
+                    aph ^= 1;
+                }
+                if (!mbar_wait(&ctl.q_full[qs], qph, ctl, a.status, row)) break;
+                if (!mbar_wait(&ctl.acc_empty[ab], abph ^ 1, ctl, a.status, row)) break;
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t d = tmem + ab * 256 + h * kCols;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int kc = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ad = sw128_desc(smem_u32(sA + kc * (kTileKeys * 128) + h * (128 * 128) + ko));
+                            const uint64_t bd = sw128_desc(smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128) + ko));
+                            mma_bf16(d, ad, bd, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&ctl.q_empty[qs]);
+                    mma_commit(&ctl.acc_full[ab]);
+                    if (flags & kLast) mma_commit(&ctl.a_empty);
+                }
+                issued = true;
+                __syncwarp();
+                if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
+                if (++ab == 2) { ab = 0; abph ^= 1; }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.m_empty[mk]);
+            if (++mk == kMeta) { mk = 0; mph ^= 1; }
+        }
+        // all MMAs issued by this thread are complete before TMEM is released
+        if (issued) {
+            if (lane == 0) mma_commit(&ctl.drain);
+            __syncwarp();
+            const uint64_t t0 = now_ns();
+            while (!mbar_test(&ctl.drain, 0) && now_ns() - t0 < kTimeoutNs) {}
+        }
+    } else if (warp >= 2) {
+        // ============================== epilogue ==============================
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int key = half * 128 + quad * 32 + lane;  // key within the tile = TMEM lane of its half
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        uint32_t mk = 0, mph = 0, ab = 0, abph = 0;
+        float acc0 = 0.f, acc1 = 0.f;
+        int kpos = INT32_MAX, wkmin = INT32_MAX, wkmax = INT32_MIN;
+        bool kv = false;
+        for (;;) {
+            if (!mbar_wait(&ctl.m_full[mk], mph, ctl, a.status, -1)) break;
+            const Item &it = items[mk];
+            const int row = it.row;
+            if (row < 0) break;
+            const int flags = it.flags, blk = it.blk;
+            if (flags & kFirst) {
+                acc0 = acc1 = 0.f;
+                kv = (it.kvalid[key >> 5] >> (key & 31)) & 1u;
+                kpos = it.kpos[key];
+                int mn = kv ? kpos : INT32_MAX, mx = kv ? kpos : INT32_MIN;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
+                wkmin = mn;
+                wkmax = mx;
+            }
+            if (blk >= 0) {
+                if (!mbar_wait(&ctl.acc_full[ab], abph, ctl, a.status, row)) break;
+                tc_fence_after();
+                const int vcols = it.valid_cols;
+                const float sc = a.scale_log2e;
+                const uint32_t tbase = tmem + lane_addr + ab * 256 + half * kCols;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    if (ch * 32 >= vcols) break;
+                    if (wkmax == INT32_MIN || it.cq_max[ch] < wkmin) continue;  // no key of this warp sees the chunk
+                    uint32_t r[32];
+                    tmem_ld32(tbase + ch * 32, r);
+                    tmem_ld_wait();
+                    const float4 *L4 = reinterpret_cast<const float4 *>(it.L + ch * 32);
+                    if ((ch + 1) * 32 <= vcols && it.cq_min[ch] >= wkmax) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 l = L4[c4];
+                            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x));
+                            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y));
+                            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z));
+                            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w));
+                        }
+                    } else {
+                        const int4 *P4 = reinterpret_cast<const int4 *>(it.qp + ch * 32);
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 l = L4[c4];
+                            const int4 p = P4[c4];
+                            const float x0 = fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x);
+                            const float x1 = fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y);
+                            const float x2 = fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z);
+                            const float x3 = fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w);
+                            acc0 += ex2(p.x >= kpos ? x0 : -INFINITY);
+                            acc1 += ex2(p.y >= kpos ? x1 : -INFINITY);
+                            acc0 += ex2(p.z >= kpos ? x2 : -INFINITY);
+                            acc1 += ex2(p.w >= kpos ? x3 : -INFINITY);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.acc_empty[ab]);
+                if (++ab == 2) { ab = 0; abph ^= 1; }
+            }
+            if (flags & kLast) {
+                if (kv) {
+                    float *dst = a.scores + (int64_t)row * c.max_slots + (int64_t)it.tile * kTileKeys + key;
+                    const float v = acc0 + acc1;
+                    *dst = a.accumulate ? *dst + v : v;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.m_empty[mk]);
+            if (++mk == kMeta) { mk = 0; mph ^= 1; }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+template <int D>
+cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool accumulate, int32_t *status,
+                     cudaStream_t stream, char *err, size_t errlen) {
+    using PL = Plan<D>;
+    auto enc = encode_fn();
+    if (!enc) {
+        snprintf(err, errlen, "cuTensorMapEncodeTiled unavailable");
+        return cudaErrorNotSupported;
+    }
+    const int G = q.group;
+    const int nqb = kCols / G;
+    if ((q.max_q + nqb - 1) / nqb > kMaxBlocks) {
+        snprintf(err, errlen, "query set too large for one pass: max_q %d > %d", q.max_q, kMaxBlocks * nqb);
+        return cudaErrorInvalidValue;
+    }
+    CUtensorMap tk, tq;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.num_pages * 16};
+        cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+        cuuint32_t box[2] = {64, 16};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(c.k_pool), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            snprintf(err, errlen, "K tensor map encode failed (%d)", (int)r);
+            return cudaErrorInvalidValue;
+        }
+    }
+    {
+        cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)q.num_q_heads, (cuuint64_t)q.max_q,
+                              (cuuint64_t)c.num_seqs * c.num_layers};
+        cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)q.num_q_heads * D * 2,
+                                 (cuuint64_t)q.max_q * q.num_q_heads * D * 2};
+        cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)nqb, 1};
+        cuuint32_t es[4] = {1, 1, 1, 1};
+        CUresult r = enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q.q), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            snprintf(err, errlen, "Q tensor map encode failed (%d)", (int)r);
+            return cudaErrorInvalidValue;
+        }
+    }
+    TcArgs args;
+    args.c = c;
+    args.q = q;
+    args.scores = scores;
+    args.status = status;
+    args.accumulate = accumulate ? 1 : 0;
+    args.nqb = nqb;
+    args.tiles_per_row = (int)((c.max_slots + kTileKeys - 1) / kTileKeys);
+    args.total_tiles = (int64_t)c.rows * args.tiles_per_row;
+    args.scale_log2e = (float)(1.4426950408889634 / std::sqrt((double)D));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(sms, args.total_tiles);
+    score_tc_kernel<D><<<grid, kThreads, PL::kBytes, stream>>>(tk, tq, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_tc(const CacheView &c, const QueryView &q, float *scores, bool accumulate, int32_t *status,
+                            cudaStream_t stream, char *err, size_t errlen) {
+    if (c.head_dim == 64) return launch_t<64>(c, q, scores, accumulate, status, stream, err, errlen);
+    return launch_t<128>(c, q, scores, accumulate, status, stream, err, errlen);
+}
+
+}  // namespace kvc

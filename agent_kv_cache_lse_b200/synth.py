@@ -358,3 +358,30 @@ def logits(spec: Spec, s: int, step0: int, steps: int, device="cpu") -> torch.Te
     v = torch.arange(spec.vocab, device=device, dtype=torch.int64)
     c = (s * (1 << 24) + t[:, None]) * (1 << 20) + v[None, :]
     return normal(spec.seed, S_LOGITS, c, sigma=spec.logits_sigma)
+
+
+def streaming_queries(spec: Spec, n_total: Sequence[int], device="cpu") -> Queries:
+    """Beacon plus recent query set at the current decode position of each sequence.
+
+    Beacons (INT32_MAX position, unmasked) are fixed per (seq, layer, q head, index);
+    the recent queries are the last `num_recent` decoded tokens, drawn by position.
+    """
+    S, L, Hq, D = spec.num_seqs, spec.num_layers, spec.num_q_heads, spec.head_dim
+    nb, nr = spec.num_beacons, spec.num_recent
+    max_q = nb + nr
+    q = torch.zeros((S, L, max_q, Hq, D), dtype=torch_dtype(spec), device=device)
+    q_pos = torch.full((S, max_q), 2**31 - 1, dtype=torch.int32)
+    hh = torch.arange(Hq, device=device, dtype=torch.int64)
+    d = torch.arange(D, device=device, dtype=torch.int64)
+    for s in range(S):
+        n = int(n_total[s])
+        rec = torch.arange(n - nr, n, dtype=torch.int64)
+        q_pos[s, nb:] = rec.to(torch.int32)
+        for l in range(L):
+            jb = torch.arange(nb, device=device, dtype=torch.int64)
+            cb = counter(s, l, hh[None, :, None], jb[:, None, None], d[None, None, :])
+            q[s, l, :nb] = normal(spec.seed, S_BEACON, cb).to(torch_dtype(spec))
+            cr = counter(s, l, hh[None, :, None], rec.to(device)[:, None, None], d[None, None, :])
+            q[s, l, nb:] = normal(spec.seed, S_RECENT, cr).to(torch_dtype(spec))
+    num_q = torch.full((S,), max_q, dtype=torch.int32)
+    return Queries(q=q, q_pos=q_pos.to(device), num_q=num_q.to(device), max_q=max_q)

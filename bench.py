@@ -1,0 +1,428 @@
+"""Benchmark of the eviction/compaction hot path on B200.
+
+One step = one full eviction round (confidence ratchet -> score from LSE -> LRFU -> top-budget
+select -> slot plan -> in-place compaction) over the Llama-3-8B-shaped single layer at 32K
+context (32 q / 8 KV heads, head_dim 128, bf16, 16-token pages, ~608 action-token queries,
+budget 512, 64 decode steps of 128,256-token logits for the ratchet).  Inputs are seeded
+synthetic data resident in HBM; the compacted state is restored and L2 is flushed (a 256 MB
+write) outside the timed region before every step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  N > 1 runs one independent replica per GPU (weak scaling:
+the path shards by sequence and needs no collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV entries scored+compacted/sec at 32K ctx"
+UNIT = "entries/s"
+WORKLOAD = ("Llama-3-8B-shaped single layer: 32 q / 8 KV heads, head_dim 128, bf16 K/V ~N(0,1) with 2% "
+            "heavy-hitter keys (x4), 32,768 tokens in 16-token pages (shuffled pool), observation/reasoning/"
+            "action segments, all action tokens as queries, budget 512, ratchet over 64 steps x 128,256 logits")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def algorithmic_work(spec, layout, queries):
+    """FLOP of the QK^T contraction over visible (key, query-head) pairs, exps, and bytes of one round."""
+    P, D = spec.page_size, spec.head_dim
+    G = spec.group
+    flops = exps = 0
+    qpos = queries.q_pos.cpu().numpy()
+    numq = queries.num_q.cpu().numpy()
+    sp = layout.slot_pos.numpy()
+    entries = 0
+    for r in range(spec.rows):
+        s, _, _ = spec.row_coords(r)
+        n = int(layout.row_len[r])
+        entries += n
+        qp = np.sort(qpos[s, :numq[s]])
+        vis = G * (len(qp) - np.searchsorted(qp, sp[r, :n], side="left"))
+        flops += 2 * D * int(vis.sum())
+        exps += int(vis.sum())
+    esize = 2 if spec.dtype == "bf16" else 4
+    nq_total = int(numq.sum())
+    kv_bytes = entries * D * esize                                  # K read once by scoring
+    meta = entries * (4 + 4 + 4 + 4 + 1 + 1)                        # scores w/r, crf r/w, pos r, keep w
+    q_bytes = nq_total * spec.num_layers * spec.num_q_heads * (D * esize + 4)
+    logits = spec.num_seqs * spec.logits_steps * spec.vocab * 4
+    return dict(entries=entries, flops=flops, exps=exps, kv_bytes=kv_bytes, meta_bytes=meta, q_bytes=q_bytes,
+                logits_bytes=logits)
+
+
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx.append(float(p[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def build_workload(device):
+    from agent_kv_cache_lse_b200 import kvc, synth
+    spec = synth.llama8b_layer()
+    layout = synth.make_layout(spec)
+    kp = synth.fill_pool(spec, layout, "k", device)
+    vp = synth.fill_pool(spec, layout, "v", device)
+    qs = synth.make_queries(spec, device)
+    lse = torch.zeros((1, 1, spec.num_q_heads, qs.max_q), dtype=torch.float32, device=device)
+    cache = kvc.Cache(kp, vp, layout.block_table.to(device), layout.row_len.to(device), layout.slot_pos.to(device),
+                      layout.slot_label.to(device), 1, 1, spec.num_kv_heads)
+    queries = kvc.QuerySet(qs.q, lse, qs.q_pos.to(device), qs.num_q.to(device))
+    # the attention kernel's LSE byproduct, produced here by the library's own LSE pass (setup, untimed)
+    kvc.kvc_query_lse(cache, queries)
+    logits = torch.stack([synth.logits(spec, 0, 0, spec.logits_steps, device=device)])
+    torch.cuda.synchronize()
+    return spec, layout, cache, queries, logits
+
+
+def run_ours(args, rank, world, device):
+    from agent_kv_cache_lse_b200 import kvc
+    from agent_kv_cache_lse_b200.round import EvictionRound
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    spec, layout, cache, queries, logits = build_workload(device)
+    work = algorithmic_work(spec, layout, queries)
+    rnd = EvictionRound(cache)
+    mutable = [cache.k_pool, cache.v_pool, cache.block_table, cache.row_len, cache.slot_pos, cache.slot_label,
+               rnd.crf]
+    pristine = [t.clone() for t in mutable]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def restore():
+        for t, p in zip(mutable, pristine):
+            t.copy_(p)
+        rnd.reset_ratchet()
+        flush.fill_(1.0)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        kvc.kvc_confidence_ratchet(logits, rnd.state, rnd.budget, rnd.params, None, rnd.status)
+        if e is not None:
+            e[1].record(stream)
+        kvc.kvc_score_from_lse(cache, queries, rnd.scores, 0, rnd.status)
+        if e is not None:
+            e[2].record(stream)
+        kvc.kvc_lrfu_update(cache, rnd.scores, rnd.crf, 0.5, 0.9, 1, 0, rnd.status)
+        kvc.kvc_select_budget(cache, rnd.crf, rnd.budget, rnd.keep, rnd.kept, 0, rnd.status)
+        kvc.kvc_plan_slots(cache, rnd.keep, rnd.kept, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.status)
+        kvc.kvc_compact_pages(cache, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.kept, rnd.crf, rnd.freed,
+                              rnd.num_freed, rnd.workspace, rnd.status)
+        if e is not None:
+            e[3].record(stream)
+
+    for _ in range(args.warmup):
+        restore()
+        step()
+    torch.cuda.synchronize()
+    code = rnd.device_status()[0]
+    if code != 0:
+        raise RuntimeError(f"device status {rnd.device_status()} during warm-up")
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    local = torch.cuda.current_device()
+    ids = [x for x in vis.split(",") if x.strip().isdigit()]
+    clocks = ClockSampler(int(ids[local]) if local < len(ids) else local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        restore()
+        step(ev[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = [ev[k][0].elapsed_time(ev[k][3]) for k in range(args.steps)]
+    score_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
+    ratchet_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert rnd.device_status()[0] == 0
+
+    # end to end through the same public calls with host buffers: H2D inputs, path, D2H results
+    e2e = None
+    if rank == 0:
+        e2e = run_e2e(args, spec, cache, queries, logits, rnd, pristine, device)
+
+    cpu = cpu_baseline(spec) if (rank == 0 and world == 1 and not args.no_cpu) else None
+    if rank != 0:
+        return None
+    ms_step = total_ms / args.steps
+    value = work["entries"] * world / (total_ms / 1e3 / args.steps)
+    score_avg = float(np.mean(score_ms))
+    achieved = work["flops"] / (score_avg / 1e3) / 1e12
+    bytes_step = work["kv_bytes"] + work["meta_bytes"] + work["q_bytes"] + work["logits_bytes"]
+    t_roof = max(work["flops"] / (tf_burst * 1e12), bytes_step / (hbm * 1e9))
+    sm_mhz = (clk or {}).get("sm_mhz", 1965.0)
+    exp_ceiling = 16 * 148 * sm_mhz * 1e6
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter-based generator; shapes of the agent-trace workload)",
+        "config": {"workload": WORKLOAD, "entries_per_step": work["entries"], "rows": spec.rows,
+                   "queries": int(queries.num_q.sum()), "budget": spec.budget, "seq_len": 32768,
+                   "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before every step"},
+        "roofline": {"kernel": "score_tc_kernel (kvc_score_from_lse)", "bound": "tensor", "achieved": achieved,
+                     "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 dense (burst)", "flops_per_launch": work["flops"],
+                     "ms_per_launch": score_avg,
+                     "exp_rate_per_s": work["exps"] / (score_avg / 1e3),
+                     "exp_frac_of_mufu": work["exps"] / (score_avg / 1e3) / exp_ceiling},
+        "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_step * 1e3, "frac": t_roof / (ms_step / 1e3),
+                          "bytes_per_step": bytes_step, "flops_per_step": work["flops"], "hbm_peak_gbs": hbm},
+        "breakdown_ms": {"ratchet": float(np.mean(ratchet_ms)), "score": score_avg,
+                         "lrfu+select+plan+compact": float(np.mean(step_ms) - np.mean(score_ms) - np.mean(ratchet_ms))},
+        "gpu_launches": EvictionRound_KERNELS * args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    return line
+
+
+EvictionRound_KERNELS = 8
+
+
+def run_e2e(args, spec, cache, queries, logits, rnd, pristine, device):
+    from agent_kv_cache_lse_b200 import kvc
+    from agent_kv_cache_lse_b200.round import EvictionRound
+    # host (pinned) copies of every input of a round
+    h_in = {
+        "k": pristine[0].cpu().pin_memory(), "v": pristine[1].cpu().pin_memory(),
+        "bt": pristine[2].cpu().pin_memory(), "rl": pristine[3].cpu().pin_memory(),
+        "sp": pristine[4].cpu().pin_memory(), "sl": pristine[5].cpu().pin_memory(),
+        "q": queries.q.cpu().pin_memory(), "lse": queries.lse.cpu().pin_memory(),
+        "qpos": queries.q_pos.cpu().pin_memory(), "numq": queries.num_q.cpu().pin_memory(),
+        "logits": logits.cpu().pin_memory(),
+    }
+    d = {k: torch.empty_like(v, device=device) for k, v in h_in.items()}
+    c2 = kvc.Cache(d["k"], d["v"], d["bt"], d["rl"], d["sp"], d["sl"], 1, 1, spec.num_kv_heads)
+    q2 = kvc.QuerySet(d["q"], d["lse"], d["qpos"], d["numq"])
+    r2 = EvictionRound(c2)
+    outs = {"k": d["k"], "v": d["v"], "bt": d["bt"], "rl": d["rl"], "sp": d["sp"], "sl": d["sl"], "crf": r2.crf,
+            "freed": r2.freed, "num_freed": r2.num_freed, "budget": r2.budget}
+    h_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs.values())
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k, v in h_in.items():
+            d[k].copy_(v, non_blocking=True)
+        r2.crf.zero_()
+        r2.reset_ratchet()
+        r2.run(q2, d["logits"])
+        for k, v in outs.items():
+            h_out[k].copy_(v, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    entries = int(h_in["rl"].sum())
+    return {"value": entries / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms}
+
+
+def oracle_sample(spec, layout, kpool_rows, qrows, lse_rows, logits_np, rows, steps):
+    """The oracle's path on a sample: the given rows scored, gated, selected, planned and compacted, plus
+    `steps` decode steps of the confidence monitor.  Returns entries processed."""
+    from oracle import path as opath
+    P = spec.page_size
+    entries = 0
+    for r in rows:
+        n = int(layout.row_len[r])
+        kf, kb, vb = kpool_rows[r]
+        q, qp = qrows[r]
+        pos = layout.slot_pos[r].numpy()
+        s = opath.scores_from_lse(q, kf, qp, pos[:n], lse_rows[r])
+        crf = opath.lrfu_update(np.zeros(n), s, pos[:n], 0.5, 0.9)
+        keep = opath.select_budget(crf, pos[:n], spec.budget)
+        src, dst, m = opath.plan_slots(keep, n)
+        row = opath.PagedRow(block_table=np.arange(kb.shape[0]), n=n, slot_pos=pos.copy(),
+                             slot_label=layout.slot_label[r].numpy().copy(), crf=crf)
+        opath.compact_row(kb, vb, row, src, dst, m, P)
+        entries += n
+    rt = opath.Ratchet()
+    rt.round(logits_np[:steps])
+    return entries
+
+
+def prepare_oracle_sample(spec, rows, steps):
+    """Host inputs of the oracle's sample, drawn from the seeded generator (no device involved): the rows'
+    keys, values and query set, their LSE (oracle, untimed) and `steps` decode steps of logits."""
+    from agent_kv_cache_lse_b200 import synth
+    from oracle import path as opath
+    P, G = spec.page_size, spec.group
+    layout = synth.make_layout(spec)
+    qs = synth.make_queries(spec, "cpu")
+    kpool_rows, qrows, lse_rows = {}, {}, {}
+    for r in rows:
+        s, l, h = spec.row_coords(r)
+        n = int(layout.row_len[r])
+        pos = layout.slot_pos[r, :n].to(torch.int64)
+        k = synth.key_values(spec, s, l, h, pos, "k")
+        v = synth.key_values(spec, s, l, h, pos, "v")
+        npg = -(-n // P)
+        kb = torch.zeros((npg * P, spec.head_dim), dtype=k.dtype)
+        vb = torch.zeros_like(kb)
+        kb[:n], vb[:n] = k, v
+        kpool_rows[r] = (k.to(torch.float64).numpy(), kb.view(npg, P, -1).view(torch.int16).numpy(),
+                         vb.view(npg, P, -1).view(torch.int16).numpy())
+        nq = int(qs.num_q[s])
+        q = qs.q[s, l, :nq, h * G:(h + 1) * G].to(torch.float64).numpy()
+        qp = qs.q_pos[s, :nq].numpy()
+        qrows[r] = (q, qp)
+        lse_rows[r] = opath.attention_lse(q, kpool_rows[r][0], qp, pos.numpy()).astype(np.float32).astype(np.float64)
+    lg = synth.logits(spec, 0, 0, steps, device="cpu").numpy().astype(np.float64)
+    return layout, (kpool_rows, qrows, lse_rows, lg)
+
+
+def cpu_baseline(spec, rows=(0, 3, 7), steps=24):
+    layout, prep = prepare_oracle_sample(spec, list(rows), steps)
+    t0 = time.perf_counter()
+    entries = oracle_sample(spec, layout, *prep, list(rows), steps)
+    dt = time.perf_counter() - t0
+    return {"value": entries / dt, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{len(rows)} of {spec.rows} rows ({entries} entries) through score/LRFU/select/plan/compact "
+                      f"plus {steps} of 64 ratchet steps (the rows' share of the round's monitor work); "
+                      f"{dt:.1f} s of CPU time; LSE prepared untimed",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is one row of the workload through the whole path plus
+    8 of the 64 ratchet steps (its share), on the host cores."""
+    if rank != 0:
+        return None
+    from agent_kv_cache_lse_b200 import synth
+    spec = synth.llama8b_layer()
+    rows = [0]
+    layout, prep = prepare_oracle_sample(spec, rows, 8)
+    for _ in range(args.warmup):
+        oracle_sample(spec, layout, *prep, rows, 8)
+    t0 = time.perf_counter()
+    entries = 0
+    for _ in range(args.steps):
+        entries += oracle_sample(spec, layout, *prep, rows, 8)
+    dt = time.perf_counter() - t0
+    value = entries / dt
+    cores = len(os.sched_getaffinity(0))
+    sample = f"1 of {spec.rows} rows (32,768 entries) + 8 of 64 ratchet steps per step"
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", torch.cuda.current_device())
+    from agent_kv_cache_lse_b200 import kvc
+    kvc.lib()   # raises if the CUDA library is missing
+    line = run_ours(args, rank, world, device)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,275 @@
+/*
+ * kvc.h -- C ABI of libkvc: attention-guided KV-cache eviction and in-place paged
+ * compaction on NVIDIA B200 (sm_100a).
+ *
+ * The path has five steps, each an entry point below:
+ *   1. kvc_score_from_lse      score every cached entry by the attention it receives
+ *                              from a query set, recovered from the attention
+ *                              log-sum-exp ("ActKV Dissected", Component 3 and
+ *                              Component 1; "BeaconKV", Key ideas, for beacon plus
+ *                              recent queries)
+ *   2. kvc_lrfu_update         fold the action-critical hit signal into an LRFU
+ *                              combined recency-frequency value, lambda = 0.5
+ *                              ("ActKV Dissected", Component 1)
+ *   3. kvc_confidence_ratchet  top-20 average-NLL confidence monitor, min-pooled
+ *                              (window 64, stride 8), linear-fit slope, one-way
+ *                              x1.75 budget ratchet from 512 to 30,000
+ *                              ("ActKV Dissected", Summary, Component 2, Lineage)
+ *      kvc_select_budget       keep the top-budget entries per row, ties broken by
+ *                              lower token position
+ *   4. kvc_plan_slots          conflict-free slot plan: survivors outside the target
+ *                              region paired one-to-one with holes inside it
+ *                              ("ActKV Dissected", Component 3)
+ *   5. kvc_compact_pages       one parallel in-place copy pass; shrunk block table
+ *                              and freed-page list ("ActKV Dissected", Component 3)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer inside the structures and every array argument is DEVICE memory
+ *   owned by the caller, unless stated otherwise.  The library never allocates,
+ *   frees or synchronises; it keeps no state between calls except a thread-local
+ *   last-error string.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * - Errors the host can see (null pointers, unsupported dtype or head_dim, sizes)
+ *   return a status other than KVC_OK before anything is enqueued.
+ *   kvc_last_error() then describes the problem.
+ * - Errors only the device can see (a page id outside the pool, a row length over
+ *   capacity, a non-finite value, a full freed list, a wait that gave up) are
+ *   written to `d_status` when it is not NULL: d_status points to two device
+ *   int32 values {code, row}, which the caller zeroes; the first error wins and
+ *   later ones are dropped.  The offending row is skipped; no kernel traps.  The
+ *   caller reads d_status after synchronising.
+ * - A "row" is one (sequence, layer, KV head) stream of cached entries:
+ *       row = (seq * num_layers + layer) * num_kv_heads + kv_head.
+ *   Its logical slots are 0 .. row_len[row]-1; slot i lives in physical page
+ *   block_table[row][i / page_size] at offset i % page_size.
+ * - Inputs are not modified except the arrays documented as in/out.
+ * - Calls on disjoint buffers may run concurrently on different streams.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvc_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    KVC_OK = 0,
+    KVC_ERR_INVALID_ARGUMENT = 1, /* null pointer, size out of range, inconsistent shapes */
+    KVC_ERR_UNSUPPORTED = 2,      /* valid but not implemented (dtype, head_dim, page_size) */
+    KVC_ERR_CUDA = 3,             /* a CUDA runtime call failed (launch, attribute, tensor map) */
+    KVC_ERR_DEVICE_FAULT = 4,     /* reserved for callers that fold d_status into a kvc_status */
+    KVC_ERR_TIMEOUT = 5           /* reserved for callers that fold d_status into a kvc_status */
+} kvc_status;
+
+/* codes written to d_status[0] by kernels */
+#define KVC_DEV_OK 0
+#define KVC_DEV_BAD_PAGE 1       /* page id outside [0, num_pages), or -1 inside a row's length */
+#define KVC_DEV_BAD_LENGTH 2     /* row_len < 0 or > max_pages_per_row * page_size, or new length > row_len */
+#define KVC_DEV_NONFINITE 3      /* NaN or +inf in an LSE, score, CRF or logit */
+#define KVC_DEV_KEPT_MISMATCH 4  /* kept[row] differs from the number of set bytes in keep */
+#define KVC_DEV_FREED_OVERFLOW 5 /* freed list longer than freed_capacity */
+#define KVC_DEV_BAD_MOVE 6       /* a move outside [0, row_len) or not hole/survivor */
+#define KVC_DEV_TIMEOUT 7        /* a bounded wait inside a kernel gave up */
+
+typedef enum { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
+
+/*
+ * The paged cache (layout adopted for per-KV-head eviction: a page holds
+ * page_size tokens of ONE (layer, KV head) row, so rows compact independently).
+ *   k_pool, v_pool  [num_pages][page_size][head_dim] of `dtype`, same page ids;
+ *                   16-byte aligned.  In/out for kvc_compact_pages only.
+ *   block_table     [rows][max_pages_per_row] int32, -1 = no page.  In/out for compaction.
+ *   row_len         [rows] int32.  In/out for compaction.
+ *   slot_pos        [rows][max_pages_per_row * page_size] int32: the original token
+ *                   position of each logical slot (order after compaction is not
+ *                   position order).  In/out for compaction.
+ *   slot_label      same shape, uint8: 0 observation, 1 reasoning, 2 action; may be
+ *                   NULL.  In/out for compaction.
+ */
+typedef struct {
+    void *k_pool;
+    void *v_pool;
+    int64_t num_pages;
+    int32_t page_size;
+    int32_t head_dim;
+    int32_t dtype; /* kvc_dtype */
+    int32_t max_pages_per_row;
+    int32_t *block_table;
+    int32_t *row_len;
+    int32_t *slot_pos;
+    uint8_t *slot_label;
+    int32_t num_seqs;
+    int32_t num_layers;
+    int32_t num_kv_heads;
+    int32_t reserved;
+} kvc_cache;
+
+/*
+ * The query set of one round (action-region tokens, or beacon plus recent queries).
+ *   q      [num_seqs][num_layers][max_q][num_q_heads][head_dim], the cache's dtype,
+ *          16-byte aligned.  Query head h belongs to KV head h / (num_q_heads / num_kv_heads).
+ *   lse    [num_seqs][num_layers][num_q_heads][max_q] fp32, natural log of the softmax
+ *          denominator of each query column over the keys it attended to.  Input to
+ *          scoring; output of kvc_query_lse.  -inf marks a column that saw no key.
+ *   q_pos  [num_seqs][max_q] int32 token position of each query (causal mask: a query
+ *          sees keys whose slot_pos <= q_pos); INT32_MAX marks an unmasked beacon.
+ *   num_q  [num_seqs] int32 number of valid queries (the first num_q[seq] of max_q).
+ */
+typedef struct {
+    const void *q;
+    float *lse;
+    const int32_t *q_pos;
+    const int32_t *num_q;
+    int32_t max_q;
+    int32_t num_q_heads;
+} kvc_queries;
+
+/* flags of kvc_score_from_lse */
+#define KVC_SCORE_ACCUMULATE 1u  /* add into scores instead of overwriting them */
+#define KVC_SCORE_COMPUTE_LSE 2u /* run kvc_query_lse first (beacons have no decode-time LSE) */
+#define KVC_SCORE_SIMT 4u        /* force the CUDA-core path even for bf16 (cross-check) */
+
+/* flags of kvc_lrfu_update */
+#define KVC_HIT_BINARY 1u /* a hit counts 1 instead of its attention score */
+
+typedef struct {
+    int32_t top_k;      /* tokens averaged per step: 20 */
+    int32_t window;     /* min-pool window: 64 */
+    int32_t stride;     /* min-pool stride: 8 */
+    int32_t grow_num;   /* growth factor numerator: 7  (7/4 = 1.75) */
+    int32_t grow_den;   /* growth factor denominator: 4 */
+    int32_t init_budget;/* 512 */
+    int32_t cap;        /* 30000 */
+    int32_t min_points; /* pooled points needed before a fit: 2 */
+    int32_t max_steps;  /* largest `steps` of one kvc_confidence_ratchet call (sizes the state) */
+    int32_t reserved;
+} kvc_ratchet_params;
+
+/* Per-sequence ratchet state as laid out in the state buffer (documented so that a
+ * caller can snapshot, restore or inspect it).  The buffer holds num_seqs of these,
+ * then num_seqs histories of (window - 1 + max_steps) floats. */
+typedef struct {
+    int64_t steps_seen;       /* decode steps consumed so far */
+    int64_t last_expand_step; /* steps_seen at the last expansion (0 before any) */
+    int64_t next_window;      /* index of the first pooled window not yet emitted */
+    double fit_n, fit_sx, fit_sy, fit_sxy, fit_sxx; /* OLS sums since the last expansion */
+    double last_slope;        /* slope of the last evaluation, NaN when none was made */
+    int32_t budget;
+    int32_t expansions;
+    int32_t last_points;      /* pooled points in the last fit */
+    int32_t reserved;
+} kvc_ratchet_seq_state;
+
+const char *kvc_status_string(kvc_status status);
+const char *kvc_last_error(void);
+int32_t kvc_version(void);
+
+/*
+ * Step 1 (input of): natural-log LSE of every valid query column over the keys it
+ * sees in its row (causal by slot_pos; beacons see all keys), written to queries->lse.
+ * Stands in for the LSE a paged-attention kernel emits beside its output
+ * ("ActKV Dissected", Component 3); needed for beacon queries, which no attention
+ * produced ("BeaconKV", Key ideas).  Columns that see no key get -inf.
+ */
+kvc_status kvc_query_lse(const kvc_cache *cache, const kvc_queries *queries, int32_t *d_status,
+                         kvc_stream_t stream);
+
+/*
+ * Step 1: scores[row][slot] = sum over valid queries j of the row's sequence and layer,
+ * and over the query heads g of the row's GQA group, of
+ *     [q_pos_j >= slot_pos] * exp(q_{j,g} . k_slot / sqrt(head_dim) - lse_{j,g}).
+ * scores: [rows][max_pages_per_row * page_size] fp32, written for slots < row_len only.
+ * bf16 caches run on the tensor cores (tcgen05, TMA page gather); fp32 caches on CUDA
+ * cores in fp32.  Requires page_size 16 and head_dim 64 or 128 for bf16.
+ */
+kvc_status kvc_score_from_lse(const kvc_cache *cache, const kvc_queries *queries, float *scores,
+                              uint32_t flags, int32_t *d_status, kvc_stream_t stream);
+
+/*
+ * Step 2: per row, the hit signal is the row's action-critical entries -- the shortest
+ * prefix of the order (score descending, slot_pos ascending, slot ascending) whose mass
+ * reaches hit_mass * (total score) -- and then
+ *     crf[row][slot] <- h + 2^(-lambda * dt_rounds) * crf[row][slot]
+ * with h = score (or 1 with KVC_HIT_BINARY) for hits and 0 otherwise.  hit_mass >= 1
+ * turns the gate off (every entry with a positive score is a hit).  crf is in/out,
+ * [rows][max_slots] fp32, updated for slots < row_len.
+ */
+kvc_status kvc_lrfu_update(const kvc_cache *cache, const float *scores, float *crf, float lambda,
+                           float hit_mass, int32_t dt_rounds, uint32_t flags, int32_t *d_status,
+                           kvc_stream_t stream);
+
+/*
+ * Step 3 (selection): keep[row][slot] = 1 for the first min(budget[seq], row_len) slots of
+ * the order (crf descending, slot_pos ascending, slot ascending), 0 for the rest of the
+ * row.  Entries whose label bit is set in protect_label_mask are always kept and use up
+ * budget first.  kept[row] = number kept.  budget is [num_seqs] int32 on the device
+ * (the ratchet's output).  keep: [rows][max_slots] uint8 (written for slots < row_len).
+ */
+kvc_status kvc_select_budget(const kvc_cache *cache, const float *crf, const int32_t *budget,
+                             uint32_t protect_label_mask, uint8_t *keep, int32_t *kept,
+                             int32_t *d_status, kvc_stream_t stream);
+
+/*
+ * Step 4: with m = kept[row], the holes are the slots i < m with keep 0 and the
+ * survivors are the slots i >= m with keep 1, both ascending; move j copies survivor j
+ * into hole j.  move_src/move_dst: [rows][max_slots] int32 (first num_moves[row] valid).
+ * No slot is written twice and no destination is a source, so one parallel pass is safe.
+ */
+kvc_status kvc_plan_slots(const kvc_cache *cache, const uint8_t *keep, const int32_t *kept,
+                          int32_t *move_src, int32_t *move_dst, int32_t *num_moves,
+                          int32_t *d_status, kvc_stream_t stream);
+
+/* bytes of device workspace kvc_compact_pages needs for `rows` rows */
+size_t kvc_compact_workspace_bytes(int32_t rows);
+
+/*
+ * Step 5: for every move, copy the K and V vectors and slot_pos, slot_label and (when
+ * crf is not NULL) crf from the source slot to the destination slot, in place.  Then,
+ * with m = new_len[row] (the kept count) and n = row_len[row]: the row's logical pages
+ * ceil(m/P) .. ceil(n/P)-1 are appended to `freed` (rows in order, pages ascending
+ * within a row) and set to -1 in the block table, and row_len[row] = m.
+ * freed: [freed_capacity] int32; *num_freed (device int64) = total freed.  Source slots
+ * are not cleared.  workspace: at least kvc_compact_workspace_bytes(rows) bytes of
+ * device memory whose contents need not be preserved between calls.
+ */
+kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, const int32_t *move_dst,
+                             const int32_t *num_moves, const int32_t *new_len, float *crf,
+                             int32_t *freed, int64_t freed_capacity, int64_t *num_freed,
+                             void *workspace, size_t workspace_bytes, int32_t *d_status,
+                             kvc_stream_t stream);
+
+/* bytes of the ratchet state buffer for num_seqs sequences */
+size_t kvc_ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params *params);
+
+/* zero the state and set budget[seq] = state budget = params->init_budget */
+kvc_status kvc_ratchet_init(void *state, int32_t *budget, int32_t num_seqs,
+                            const kvc_ratchet_params *params, kvc_stream_t stream);
+
+/*
+ * Step 3 (monitor and ratchet), once per round: for each sequence and each of `steps`
+ * decode steps, c_t = LSE(z_t) - mean of the top_k largest z_t (the average negative
+ * log-probability of the top-k tokens).  Windows [stride*j, stride*j + window) over the
+ * sequence's step stream (continuing across calls) are min-pooled as they complete;
+ * pooled points whose window starts at or after the last expansion enter a least-squares
+ * line y = a + b*j.  After the round, if at least min_points points are in the fit and
+ * b < 0, budget <- min(floor(budget * grow_num / grow_den), cap), the fit restarts, and
+ * the expansion step is recorded.  The budget never shrinks.
+ * logits: [num_seqs][steps][vocab] fp32.  budget: [num_seqs] int32 (written).
+ * confidence_out: [num_seqs][steps] fp32 c_t, or NULL.
+ */
+kvc_status kvc_confidence_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab,
+                                  void *state, int32_t *budget, float *confidence_out,
+                                  const kvc_ratchet_params *params, int32_t *d_status,
+                                  kvc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */

@@ -45,7 +45,7 @@ def logits(q: np.ndarray, k: np.ndarray) -> np.ndarray:
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     D = q.shape[-1]
-    return np.einsum("jgd,id->gji", q, k) / math.sqrt(D)
+    return np.einsum("jgd,id->gji", q, k, optimize=True) / math.sqrt(D)
 
 
 def visible(q_pos: np.ndarray, k_pos: np.ndarray) -> np.ndarray:

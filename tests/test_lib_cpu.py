@@ -1,0 +1,106 @@
+"""CPU-only checks of the C-ABI library and the host logic (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from agent_kv_cache_lse_b200 import kvc, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    with open(os.path.join(ROOT, "include", "kvc.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kvc_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_entry_point():
+    L = kvc.lib()
+    names = declared_entry_points()
+    assert {"kvc_score_from_lse", "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_pages",
+            "kvc_confidence_ratchet"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/kvc.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", kvc.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (kvc_\w+)", out))
+    assert set(names) == exported, f"exports differ from the header: {set(names) ^ exported}"
+    assert set(kvc.EXPORTS) == set(names)
+
+
+def test_struct_layouts_match_header_sizes():
+    # kvc_cache: 2 pointers + int64 + 4 int32 + 4 pointers + 4 int32 (with padding) on LP64
+    assert ctypes.sizeof(kvc.KvcCache) == 2 * 8 + 8 + 4 * 4 + 4 * 8 + 4 * 4
+    assert ctypes.sizeof(kvc.KvcQueries) == 4 * 8 + 2 * 4
+    assert ctypes.sizeof(kvc.KvcRatchetParams) == 10 * 4
+    assert ctypes.sizeof(kvc.KvcRatchetSeqState) == 3 * 8 + 6 * 8 + 4 * 4
+
+
+def test_host_validation_without_gpu():
+    L = kvc.lib()
+    assert L.kvc_score_from_lse(None, None, None, 0, None, None) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert b"NULL" in L.kvc_last_error()
+    c = kvc.KvcCache()
+    c.num_seqs, c.num_layers, c.num_kv_heads = 1, 1, 1
+    c.page_size, c.max_pages_per_row, c.head_dim, c.dtype = 16, 4, 96, kvc.KVC_BF16
+    c.block_table = c.row_len = c.slot_pos = 16
+    assert L.kvc_select_budget(ctypes.byref(c), 16, 16, 0, 16, 16, None, None) == kvc.KVC_ERR_UNSUPPORTED
+    c.head_dim = 128
+    assert L.kvc_lrfu_update(ctypes.byref(c), 16, 16, ctypes.c_float(-1.0), ctypes.c_float(0.9), 1, 0, None,
+                             None) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert L.kvc_compact_pages(ctypes.byref(c), 16, 16, 16, 16, None, 16, 4, 16, 16, 0, None,
+                               None) == kvc.KVC_ERR_INVALID_ARGUMENT   # pools missing
+    p = kvc.ratchet_params()
+    assert kvc.kvc_ratchet_state_bytes(16, p) > 16 * ctypes.sizeof(kvc.KvcRatchetSeqState)
+    bad = kvc.ratchet_params(top_k=0)
+    assert kvc.kvc_ratchet_state_bytes(16, bad) == 0
+    assert kvc.kvc_compact_workspace_bytes(10) == 11 * 8
+    assert L.kvc_status_string(2) == b"unsupported"
+
+
+def test_generator_is_chunking_independent():
+    spec = synth.llama8b_layer(ctx=1024)
+    pos = torch.arange(0, 1024)
+    whole = synth.key_values(spec, 0, 0, 3, pos)
+    parts = torch.cat([synth.key_values(spec, 0, 0, 3, pos[a:a + 100]) for a in range(0, 1024, 100)])
+    assert torch.equal(whole.view(torch.int16), parts.view(torch.int16))
+    x = synth.normal(7, synth.S_Q, torch.arange(200000))
+    assert abs(float(x.mean())) < 0.01 and abs(float(x.std()) - 1.0) < 0.01
+
+
+def test_segment_trace_shape():
+    """Observation / reasoning / action segments in the ranges given, observation first; actions ~1-2%."""
+    spec = synth.llama8b_layer()
+    lab = synth.segment_labels(spec, 0, 32768).numpy()
+    assert lab[0] == synth.LABEL_OBS
+    runs = np.split(lab, np.flatnonzero(np.diff(lab)) + 1)
+    for run in runs[:-1]:
+        lo, hi = spec.seg_ranges[int(run[0])]
+        assert lo <= len(run) <= hi
+    share = float((lab == synth.LABEL_ACTION).mean())
+    assert 0.005 < share < 0.03
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "agent_kv_cache_lse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, f)) as fh:
+                    src = fh.read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, re.M), f"{f} imports the oracle"
+
+
+def test_layout_block_tables_are_disjoint():
+    spec = synth.batch16(num_seqs=3, num_layers=2, lo=300, hi=900)
+    lay = synth.make_layout(spec)
+    bt = lay.block_table.numpy()
+    used = bt[bt >= 0]
+    assert len(np.unique(used)) == len(used)
+    assert used.max() < lay.num_pages
+    for r in range(spec.rows):
+        assert (bt[r] >= 0).sum() == -(-int(lay.row_len[r]) // 16)

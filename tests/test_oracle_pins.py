@@ -381,7 +381,7 @@ def test_pin_golden(pin, golden_dir):
 MUTATIONS = [
     ("visible", ">= np.asarray(k_pos", "<= np.asarray(k_pos"),                        # reversed causal mask
     ("logits", "/ math.sqrt(D)", "/ D"),                                              # wrong scale
-    ("logits", '"jgd,id->gji"', '"jgd,id->jgi"'),                                      # transposed operand
+    ("logits", '"jgd,id->gji", q, k', '"jgd,id->gji", q[:, ::-1], k'),                  # heads of the group swapped
     ("scores_from_lse", "lse[:, a:b, None]", "lse[::-1, a:b, None]"),                 # wrong head's LSE
     ("scores_from_lse", "np.exp(l - lse", "np.exp(l + lse"),                           # sign of the LSE
     ("attention_lse", "safe + np.log(ssum)", "np.log(ssum)"),                          # dropped max shift
