@@ -130,7 +130,7 @@ struct RadixResult {
 struct RadixShared {
     unsigned int hcnt[2048];
     unsigned long long hwt[2048];
-    unsigned long long lane_w[32];
+    unsigned long long lane_w[32][32];   // per warp, per lane: weights being combined by a group leader
     uint32_t prefix, prefix_mask;
     unsigned long long above, remaining;
     uint32_t eq_count;
@@ -139,7 +139,7 @@ struct RadixShared {
 template <bool kMass, typename KeyFn, typename WeightFn, typename ValidFn>
 __device__ RadixResult radix_search_desc(int n, unsigned long long target, KeyFn key, WeightFn weight,
                                          ValidFn valid, RadixShared &sh) {
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) {
         sh.prefix = 0;
         sh.prefix_mask = 0;
@@ -171,7 +171,7 @@ __device__ RadixResult radix_search_desc(int n, unsigned long long target, KeyFn
                 const uint32_t bin = (k >> shift) & (nb - 1);
                 const unsigned peers = __match_any_sync(active, bin);
                 const int leader = __ffs(peers) - 1;
-                if (kMass) sh.lane_w[lane] = wv;
+                if (kMass) sh.lane_w[wid][lane] = wv;
                 __syncwarp(active);
                 if (lane == leader) {
                     atomicAdd(&sh.hcnt[bin], (unsigned)__popc(peers));
@@ -180,7 +180,7 @@ __device__ RadixResult radix_search_desc(int n, unsigned long long target, KeyFn
                         unsigned p = peers;
                         while (p) {
                             const int l = __ffs(p) - 1;
-                            s += sh.lane_w[l];
+                            s += sh.lane_w[wid][l];
                             p &= p - 1;
                         }
                         atomicAdd(&sh.hwt[bin], s);

@@ -373,7 +373,8 @@ def test_ratchet_rounds_parity():
         for s in range(S):
             assert st[s].budget == want[s] and st[s].expansions == orc[s].expansions
             if not math.isnan(orc[s].last_slope):
-                assert abs(st[s].last_slope - orc[s].last_slope) <= 1e-6 * (abs(orc[s].last_slope) + 1e-3)
+                # fp32 confidences against fp64: the slopes agree to ~1e-8 absolute here
+                assert abs(st[s].last_slope - orc[s].last_slope) <= 1e-6 + 1e-4 * abs(orc[s].last_slope)
     assert budget.cpu().tolist()[1] == 512
 
 
