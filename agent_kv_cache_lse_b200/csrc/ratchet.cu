@@ -14,7 +14,7 @@
 //   uses the k-th largest of the per-thread maxima as a lower bound to pick a short
 //   candidate list; when that list overflows (many equal logits) it falls back to an
 //   exact radix search over the staged slice.
-// Launch B (ratchet): one thread per sequence pools the newly completed windows,
+// Launch B (ratchet): one warp per sequence pools the newly completed windows,
 //   updates the least-squares sums, evaluates the fit once and moves the budget.
 #include <cooperative_groups.h>
 
@@ -213,8 +213,11 @@ struct UpdArgs {
     kvc_ratchet_params p;
 };
 
+// One warp per sequence: the lanes share each window's minimum and the history shift; lane 0 keeps
+// the least-squares sums and takes the decision.
 __global__ void ratchet_update_kernel(UpdArgs a) {
-    const int seq = blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int seq = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (seq >= a.num_seqs) return;
     kvc_ratchet_seq_state s = a.st[seq];
     float *h = a.hist + (int64_t)seq * a.hist_len;
@@ -225,7 +228,9 @@ __global__ void ratchet_update_kernel(UpdArgs a) {
     for (; (int64_t)R * j + W <= t1; ++j) {
         const int64_t ws = (int64_t)R * j;
         float y = INFINITY;
-        for (int64_t t = ws; t < ws + W; ++t) y = fminf(y, h[t - base]);
+        for (int64_t t = ws + lane; t < ws + W; t += 32) y = fminf(y, h[t - base]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) y = fminf(y, __shfl_xor_sync(0xffffffffu, y, o));
         if (ws >= s.last_expand_step) {
             const double x = (double)j, yy = (double)y;
             s.fit_n += 1.0;
@@ -250,11 +255,20 @@ __global__ void ratchet_update_kernel(UpdArgs a) {
             s.fit_n = s.fit_sx = s.fit_sy = s.fit_sxy = s.fit_sxx = 0.0;
         }
     }
-    // keep the last window-1 confidences for windows that straddle the next call
-    for (int k = 0; k < W - 1; ++k) h[k] = h[k + a.steps];
+    // keep the last window-1 confidences for windows that straddle the next call; chunks ascend and each
+    // reads before it writes, so the overlapping forward copy is safe
+    for (int k0 = 0; k0 < W - 1; k0 += 32) {
+        const int k = k0 + lane;
+        const float v = k < W - 1 ? h[k + a.steps] : 0.f;
+        __syncwarp();
+        if (k < W - 1) h[k] = v;
+        __syncwarp();
+    }
     s.steps_seen = t1;
-    a.st[seq] = s;
-    a.budget[seq] = s.budget;
+    if (lane == 0) {
+        a.st[seq] = s;
+        a.budget[seq] = s.budget;
+    }
 }
 
 __global__ void ratchet_init_kernel(kvc_ratchet_seq_state *st, float *hist, int32_t *budget, int32_t num_seqs,
@@ -324,7 +338,7 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
         if (e != cudaSuccess) return e;
     }
     UpdArgs u{st, hist, budget, num_seqs, steps, l.hist_len, p};
-    ratchet_update_kernel<<<(num_seqs + 63) / 64, 64, 0, stream>>>(u);
+    ratchet_update_kernel<<<(num_seqs + 3) / 4, 128, 0, stream>>>(u);
     return cudaGetLastError();
 }
 

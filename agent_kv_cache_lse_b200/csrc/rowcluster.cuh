@@ -1,0 +1,281 @@
+// Row-wide collectives for a thread-block cluster that shares one row.
+//
+// A row of up to a few tens of thousands of entries is split into C contiguous slices,
+// one per CTA of a cluster (C = 1..8).  Cluster-wide steps (a maximum, a sum, a radix
+// histogram) go through distributed shared memory: each CTA publishes its partial in a
+// double-buffered slot of its own shared memory, the cluster barrier orders the writes,
+// and every CTA reads all C slots and reduces them itself, so all CTAs reach identical
+// decisions without a broadcast.  Each collective holds exactly one cluster barrier;
+// the double buffering is safe because a slot is rewritten two collectives later, after
+// the barrier of the collective in between, which no CTA passes before finishing its
+// reads of the earlier one.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace kvc {
+
+namespace cg = cooperative_groups;
+
+constexpr int kRowBins = 256;  // 8-bit digits, 4 passes over 32-bit keys
+
+struct RowHist {
+    unsigned int cnt[kRowBins];
+    unsigned long long wt[kRowBins];
+};
+
+struct RowShared {
+    RowHist hist[2];
+    unsigned long long lane_w[32][32];  // per warp, per lane: weights combined by a group leader
+    unsigned int gcnt[kRowBins];        // cluster-wide histogram of the current pass
+    unsigned long long gwt[kRowBins];
+    // published scalars, double-buffered
+    float xf[2];
+    int xi[2][2];
+    unsigned long long xu[2];
+    // search state (the same in every CTA of the cluster)
+    uint32_t prefix, pmask;
+    unsigned long long above, remaining;
+    uint32_t eq_count;
+    int red_i[32];
+    unsigned long long red_u[32];
+    float red_f[32];
+};
+
+struct RowCtx {
+    cg::cluster_group cl;
+    int rank, nranks;
+    int par;  // collective counter (selects the buffer)
+};
+
+__device__ inline RowCtx row_ctx() {
+    RowCtx c{cg::this_cluster(), 0, 1, 0};
+    c.rank = (int)c.cl.block_rank();
+    c.nranks = (int)c.cl.num_blocks();
+    return c;
+}
+
+// Cluster-wide max of a float and OR of an int (one collective).
+__device__ inline void row_max_or(RowCtx &rc, RowShared &sh, float &v, int &flag) {
+    const float m = block_max(v, sh.red_f);
+    const int f = block_or(flag, sh.red_i);
+    const int b = rc.par & 1;
+    if (threadIdx.x == 0) {
+        sh.xf[b] = m;
+        sh.xi[b][0] = f;
+    }
+    rc.cl.sync();
+    float gm = -INFINITY;
+    int gf = 0;
+    for (int r = 0; r < rc.nranks; ++r) {
+        RowShared *p = rc.cl.map_shared_rank(&sh, r);
+        gm = fmaxf(gm, p->xf[b]);
+        gf |= p->xi[b][0];
+    }
+    rc.par++;
+    v = gm;
+    flag = gf;
+}
+
+// Cluster-wide sum of an int; also returns the sum over lower ranks (exclusive prefix).
+__device__ inline int row_sum_int(RowCtx &rc, RowShared &sh, int v, int *below) {
+    const int s = block_sum<int>(v, sh.red_i);
+    const int b = rc.par & 1;
+    if (threadIdx.x == 0) sh.xi[b][1] = s;
+    rc.cl.sync();
+    int tot = 0, low = 0;
+    for (int r = 0; r < rc.nranks; ++r) {
+        const int x = rc.cl.map_shared_rank(&sh, r)->xi[b][1];
+        tot += x;
+        if (r < rc.rank) low += x;
+    }
+    rc.par++;
+    if (below) *below = low;
+    return tot;
+}
+
+// Cluster-wide sums of two ints (CTA totals of v0, v1), with the sums over lower ranks.
+__device__ inline void row_sum_int2(RowCtx &rc, RowShared &sh, int v0, int v1, int tot[2], int below[2]) {
+    const int s0 = block_sum<int>(v0, sh.red_i);
+    const int s1 = block_sum<int>(v1, sh.red_i);
+    const int b = rc.par & 1;
+    if (threadIdx.x == 0) {
+        sh.xi[b][0] = s0;
+        sh.xi[b][1] = s1;
+    }
+    rc.cl.sync();
+    tot[0] = tot[1] = below[0] = below[1] = 0;
+    for (int r = 0; r < rc.nranks; ++r) {
+        const RowShared *p = rc.cl.map_shared_rank(&sh, r);
+        const int x0 = p->xi[b][0], x1 = p->xi[b][1];
+        tot[0] += x0;
+        tot[1] += x1;
+        if (r < rc.rank) {
+            below[0] += x0;
+            below[1] += x1;
+        }
+    }
+    rc.par++;
+}
+
+// Cluster-wide sum of an unsigned 64-bit integer.
+__device__ inline unsigned long long row_sum_u64(RowCtx &rc, RowShared &sh, unsigned long long v) {
+    const unsigned long long s = block_sum<unsigned long long>(v, sh.red_u);
+    const int b = rc.par & 1;
+    if (threadIdx.x == 0) sh.xu[b] = s;
+    rc.cl.sync();
+    unsigned long long tot = 0;
+    for (int r = 0; r < rc.nranks; ++r) tot += rc.cl.map_shared_rank(&sh, r)->xu[b];
+    rc.par++;
+    return tot;
+}
+
+// Radix search over the cluster's row, from the most significant 8-bit digit down.  Finds the key T
+// at which the running weight of the valid keys in descending key order first reaches `target`
+// (>= 1, <= total weight); weight is 1 (count mode) or a fixed-point mass (mass mode).  The slice of
+// this CTA is [lo, hi).  Same result in every thread of every CTA:
+//   key = T, above = total weight of valid keys > T, eq_count = number of valid keys == T.
+template <bool kMass, typename KeyFn, typename WeightFn, typename ValidFn>
+__device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi, unsigned long long target,
+                                      KeyFn key, WeightFn weight, ValidFn valid) {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) {
+        sh.prefix = 0;
+        sh.pmask = 0;
+        sh.above = 0;
+        sh.remaining = target;
+        sh.eq_count = 0;
+    }
+    __syncthreads();
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        const int b = rc.par & 1;
+        RowHist &h = sh.hist[b];
+        for (int i = tid; i < kRowBins; i += blockDim.x) {
+            h.cnt[i] = 0;
+            if (kMass) h.wt[i] = 0;
+        }
+        __syncthreads();
+        const uint32_t prefix = sh.prefix, pmask = sh.pmask;
+        const int span = hi - lo;
+        const int nround = (span + blockDim.x - 1) / blockDim.x * blockDim.x;
+        for (int off = tid; off < nround; off += blockDim.x) {
+            const int i = lo + off;
+            bool in = false;
+            uint32_t k = 0;
+            unsigned long long wv = 0;
+            if (off < span && valid(i)) {
+                k = key(i);
+                in = (k & pmask) == prefix;
+                if (kMass && in) wv = weight(i);
+            }
+            const unsigned active = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                const uint32_t bin = (k >> shift) & (kRowBins - 1);
+                const unsigned peers = __match_any_sync(active, bin);
+                const int leader = __ffs(peers) - 1;
+                if (kMass) sh.lane_w[wid][lane] = wv;
+                __syncwarp(active);
+                if (lane == leader) {
+                    atomicAdd(&h.cnt[bin], (unsigned)__popc(peers));
+                    if (kMass) {
+                        unsigned long long s = 0;
+                        if (peers == 0xffffffffu) {
+                            // whole warp in one bin: tree-free sum in registers of the leader
+                            for (int l = 0; l < 32; ++l) s += sh.lane_w[wid][l];
+                        } else {
+                            unsigned p = peers;
+                            while (p) {
+                                s += sh.lane_w[wid][__ffs(p) - 1];
+                                p &= p - 1;
+                            }
+                        }
+                        atomicAdd(&h.wt[bin], s);
+                    }
+                }
+                __syncwarp(active);
+            }
+        }
+        rc.cl.sync();
+        for (int i = tid; i < kRowBins; i += blockDim.x) {
+            unsigned int c = 0;
+            unsigned long long w = 0;
+            for (int r = 0; r < rc.nranks; ++r) {
+                const RowHist &rh = rc.cl.map_shared_rank(&sh, r)->hist[b];
+                c += rh.cnt[i];
+                if (kMass) w += rh.wt[i];
+            }
+            sh.gcnt[i] = c;
+            sh.gwt[i] = kMass ? w : (unsigned long long)c;
+        }
+        rc.par++;
+        __syncthreads();
+        if (tid < 32) {
+            constexpr int per = kRowBins / 32;
+            const int top = kRowBins - 1 - lane * per;  // bins top, top-1, ..., top-per+1
+            unsigned long long mine = 0;
+#pragma unroll
+            for (int q = 0; q < per; ++q) mine += sh.gwt[top - q];
+            unsigned long long incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const unsigned long long excl = incl - mine, rem = sh.remaining;
+            const bool here = excl < rem && incl >= rem;
+            const unsigned who = __ballot_sync(0xffffffffu, here);
+            if (here && lane == __ffs(who) - 1) {
+                unsigned long long run = excl;
+                for (int q = 0; q < per; ++q) {
+                    const int bin = top - q;
+                    const unsigned long long w = sh.gwt[bin];
+                    if (run + w >= rem) {
+                        sh.above += run;
+                        sh.remaining = rem - run;
+                        sh.prefix |= (uint32_t)bin << shift;
+                        sh.pmask |= (uint32_t)(kRowBins - 1) << shift;
+                        sh.eq_count = sh.gcnt[bin];
+                        break;
+                    }
+                    run += w;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    RadixResult r;
+    r.key = sh.prefix;
+    r.above = sh.above;
+    r.eq_count = sh.eq_count;
+    __syncthreads();
+    return r;
+}
+
+// Rank, in slot order over the whole row, of the entries flagged by amb(i) (contiguous chunks per
+// thread, slices in rank order); calls out(i, rank) for each flagged entry.
+template <typename AmbFn, typename OutFn>
+__device__ void row_ordered_ranks(RowCtx &rc, RowShared &sh, int lo, int hi, AmbFn amb, OutFn out) {
+    const int span = hi - lo;
+    const int chunk = (span + blockDim.x - 1) / blockDim.x;
+    const int b0 = lo + min(span, (int)threadIdx.x * chunk), b1 = lo + min(span, ((int)threadIdx.x + 1) * chunk);
+    int cnt = 0;
+    for (int i = b0; i < b1; ++i) cnt += amb(i) ? 1 : 0;
+    int total;
+    int rank = block_exclusive_scan(cnt, sh.red_i, &total);
+    int below = 0;
+    row_sum_int(rc, sh, cnt, &below);
+    rank += below;
+    for (int i = b0; i < b1; ++i)
+        if (amb(i)) out(i, rank++);
+}
+
+__host__ inline int row_cluster_size(int rows, int sms) {
+    int c = 1;
+    while (c < 8 && (int64_t)rows * c < 2 * (int64_t)sms) c <<= 1;
+    return c;
+}
+
+}  // namespace kvc

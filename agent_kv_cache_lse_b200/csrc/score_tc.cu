@@ -45,8 +45,8 @@ constexpr int kPagesPerTile = 16;       // page_size 16
 constexpr int kCols = 128;              // MMA N: query columns per block
 constexpr int kMeta = 8;                // metadata ring depth
 constexpr int kMaxBlocks = 256;         // column blocks per sequence
-constexpr int kThreads = 320;           // 10 warps
-constexpr int kEpiWarps = 8;
+constexpr int kThreads = 576;           // 18 warps
+constexpr int kEpiWarps = 16;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 struct alignas(16) Item {
@@ -63,13 +63,15 @@ constexpr int kFirst = 1, kLast = 2;
 
 struct Ctrl {
     uint64_t q_full[8], q_empty[8];
-    uint64_t a_full, a_empty;
+    uint64_t a_full[2], a_empty[2];        // double-buffered K tile
     uint64_t acc_full[2], acc_empty[2];
     uint64_t m_full[kMeta], m_empty[kMeta];
+    uint64_t part_full[2];                 // column-half partial sums of a tile, double-buffered
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort;
     int32_t blk_qmin[kMaxBlocks], blk_qmax[kMaxBlocks];
+    float part[2][kTileKeys];
 };
 
 struct TcArgs {
@@ -193,15 +195,65 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipes: x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez exchange, derived by
+// exp2_poly.py beside this file: max relative error 7.5e-5); 2^n enters through the exponent bits.
+// x is clamped at -126 so the exponent arithmetic stays in range (the result is then ~1e-38).
+__device__ __forceinline__ float exp2_fma(float x) {
+    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
+                    kC3 = 0.0551716685295105f;
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x = fmaxf(x, -126.0f);
+    const float t = x + kRound;
+    const float f = x - (t - kRound);
+    float p = fmaf(kC3, f, kC2);
+    p = fmaf(p, f, kC1);
+    p = fmaf(p, f, kC0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// One 32-column chunk of a key's accumulator row: x = acc * log2(e)/sqrt(D) - lse_col * log2(e), causal
+// select (unless every column of the chunk sees every key of the warp), 2^x, running sums.  Every
+// fourth column's exponential runs on the FMA pipes to relieve the MUFU unit.
+__device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *L, const int32_t *qp, int kpos,
+                                          float sc, bool fast, float &acc0, float &acc1) {
+    const float4 *L4 = reinterpret_cast<const float4 *>(L);
+    if (fast) {
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l = L4[c4];
+            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x));
+            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y));
+            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z));
+            acc1 += exp2_fma(fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w));
+        }
+    } else {
+        const int4 *P4 = reinterpret_cast<const int4 *>(qp);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l = L4[c4];
+            const int4 p = P4[c4];
+            const float x0 = fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x);
+            const float x1 = fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y);
+            const float x2 = fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z);
+            const float x3 = fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w);
+            acc0 += ex2(p.x >= kpos ? x0 : -INFINITY);
+            acc1 += ex2(p.y >= kpos ? x1 : -INFINITY);
+            acc0 += ex2(p.z >= kpos ? x2 : -INFINITY);
+            acc1 += ex2(p.w >= kpos ? x3 : -INFINITY);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- shared memory plan
 template <int D>
 struct Plan {
     static constexpr int kChunks = D / 64;                       // 128-byte K chunks
     static constexpr int kABytes = kTileKeys * D * 2;           // whole K tile
     static constexpr int kBBytes = kCols * D * 2;                // one Q block
-    static constexpr int kStages = D == 128 ? 4 : 8;
-    static constexpr int kOffA = 0;
-    static constexpr int kOffB = kABytes;
+    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kOffA = 0;                              // two K tiles
+    static constexpr int kOffB = 2 * kABytes;
     static constexpr int kOffItems = kOffB + kStages * kBBytes;
     static constexpr int kOffCtrl = kOffItems + kMeta * (int)sizeof(Item);
     static constexpr int kBytes = kOffCtrl + (int)sizeof(Ctrl) + 1024;  // + alignment slack
@@ -223,18 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CacheView &c = a.c;
 
     // zero the operand buffers once so rows no load ever fills hold finite values
-    for (int i = threadIdx.x; i < (PL::kABytes + PL::kStages * PL::kBBytes) / 16; i += kThreads)
+    for (int i = threadIdx.x; i < (2 * PL::kABytes + PL::kStages * PL::kBBytes) / 16; i += kThreads)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < PL::kStages; ++s) {
             mbar_init(&ctl.q_full[s], 1);
             mbar_init(&ctl.q_empty[s], 1);
         }
-        mbar_init(&ctl.a_full, 1);
-        mbar_init(&ctl.a_empty, 1);
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl.a_full[b], 1);
+            mbar_init(&ctl.a_empty[b], 1);
             mbar_init(&ctl.acc_full[b], 1);
             mbar_init(&ctl.acc_empty[b], kEpiWarps);
+            mbar_init(&ctl.part_full[b], kEpiWarps / 2);
         }
         for (int k = 0; k < kMeta; ++k) {
             mbar_init(&ctl.m_full[k], 1);
@@ -262,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================== producer ==============================
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
-        uint32_t qs = 0, qph = 0, aph = 0, mk = 0, mph = 0;
+        uint32_t qs = 0, qph = 0, mk = 0, mph = 0;
+        uint32_t ta = 0;  // K tiles loaded so far: buffer ta & 1, use (ta >> 1) of that buffer
         int cur_seq = -1, nblk = 0, nq = 0;
         const uint32_t a_tx_page = 16 * 128;                 // one 16-row, 128-byte box
         const uint32_t q_tx = (uint32_t)(G * nqb) * 128u;    // one Q box per 64-column chunk
@@ -359,17 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
                 continue;
             }
-            // K tile: one box per (page, 64-column chunk)
-            if (!mbar_wait(&ctl.a_empty, aph ^ 1, ctl, a.status, row)) { ok = false; break; }
-            aph ^= 1;
-            if (lane == 0) mbar_expect_tx(&ctl.a_full, (uint32_t)__popc(okmask) * a_tx_page * PL::kChunks);
+            // K tile into the free buffer: one box per (page, 64-column chunk)
+            const uint32_t abuf = ta & 1;
+            if (!mbar_wait(&ctl.a_empty[abuf], ((ta >> 1) & 1) ^ 1, ctl, a.status, row)) { ok = false; break; }
+            ++ta;
+            if (lane == 0) mbar_expect_tx(&ctl.a_full[abuf], (uint32_t)__popc(okmask) * a_tx_page * PL::kChunks);
             __syncwarp();
             if (page_ok) {
                 const int half = lane >> 3, r0 = (lane & 7) * 16;
 #pragma unroll
                 for (int kc = 0; kc < PL::kChunks; ++kc) {
-                    const uint32_t dst = smem_u32(sA + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
-                    tma_load_2d(dst, &tmap_k, &ctl.a_full, kc * 64, page * 16);
+                    const uint32_t dst =
+                        smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
+                    tma_load_2d(dst, &tmap_k, &ctl.a_full[abuf], kc * 64, page * 16);
                 }
             }
             // column metadata of a block: 4 columns per lane, prefetched one block ahead
@@ -465,12 +521,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t t0 = now_ns();
                 while (!mbar_test(&ctl.q_full[s], (qph ^ (s < (int)qs ? 0u : 1u)) & 1u) && now_ns() - t0 < kTimeoutNs) {}
             }
-            const uint64_t t0 = now_ns();
-            while (!mbar_test(&ctl.a_full, aph ^ 1) && now_ns() - t0 < kTimeoutNs) {}
+            for (uint32_t b = 0; b < 2; ++b) {
+                const uint32_t fills = (ta + 1 - b) / 2;  // loads that went to buffer b
+                if (fills == 0) continue;
+                const uint64_t t0 = now_ns();
+                while (!mbar_test(&ctl.a_full[b], (fills - 1) & 1) && now_ns() - t0 < kTimeoutNs) {}
+            }
         }
     } else if (warp == 1) {
         // ============================== MMA issuer ==============================
-        uint32_t qs = 0, qph = 0, aph = 0, mk = 0, mph = 0, ab = 0, abph = 0;
+        uint32_t qs = 0, qph = 0, mk = 0, mph = 0, ab = 0, abph = 0;
+        uint32_t tm = 0;  // K tiles consumed so far (same order as the producer's loads)
         bool issued = false;
         for (;;) {
             if (!mbar_wait(&ctl.m_full[mk], mph, ctl, a.status, -1)) break;
@@ -479,9 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (row < 0) break;
             const int blk = it.blk, flags = it.flags;
             if (blk >= 0) {
+                const uint32_t abuf = tm & 1;
                 if (flags & kFirst) {
-                    if (!mbar_wait(&ctl.a_full, aph, ctl, a.status, row)) break;
-                    aph ^= 1;
+                    if (!mbar_wait(&ctl.a_full[abuf], (tm >> 1) & 1, ctl, a.status, row)) break;
                 }
                 if (!mbar_wait(&ctl.q_full[qs], qph, ctl, a.status, row)) break;
                 if (!mbar_wait(&ctl.acc_empty[ab], abph ^ 1, ctl, a.status, row)) break;
@@ -493,16 +554,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const int kc = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ad = sw128_desc(smem_u32(sA + kc * (kTileKeys * 128) + h * (128 * 128) + ko));
+                            const uint64_t ad = sw128_desc(
+                                smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + h * (128 * 128) + ko));
                             const uint64_t bd = sw128_desc(smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128) + ko));
                             mma_bf16(d, ad, bd, kk > 0 ? 1u : 0u);
                         }
                     }
                     mma_commit(&ctl.q_empty[qs]);
                     mma_commit(&ctl.acc_full[ab]);
-                    if (flags & kLast) mma_commit(&ctl.a_empty);
+                    if (flags & kLast) mma_commit(&ctl.a_empty[abuf]);
                 }
                 issued = true;
+                if (flags & kLast) ++tm;
                 __syncwarp();
                 if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
                 if (++ab == 2) { ab = 0; abph ^= 1; }
@@ -520,13 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ============================== epilogue ==============================
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        // 16 warps: (TMEM lane quadrant = warp % 4, key half, column half); the two column halves of a key
+        // are added through shared memory at the end of each tile.
+        const int e = warp - 2;
+        const int quad = warp & 3, half = (e >> 2) & 1, colh = e >> 3;
         const int key = half * 128 + quad * 32 + lane;  // key within the tile = TMEM lane of its half
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        uint32_t mk = 0, mph = 0, ab = 0, abph = 0;
+        uint32_t mk = 0, mph = 0, ab = 0, abph = 0, tcount = 0;
         float acc0 = 0.f, acc1 = 0.f;
         int kpos = INT32_MAX, wkmin = INT32_MAX, wkmax = INT32_MIN;
         bool kv = false;
+        const float sc = a.scale_log2e;
         for (;;) {
             if (!mbar_wait(&ctl.m_full[mk], mph, ctl, a.status, -1)) break;
             const Item &it = items[mk];
@@ -546,57 +613,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wkmin = mn;
                 wkmax = mx;
             }
+            float *dst = a.scores + (int64_t)row * c.max_slots + (int64_t)it.tile * kTileKeys + key;
             if (blk >= 0) {
                 if (!mbar_wait(&ctl.acc_full[ab], abph, ctl, a.status, row)) break;
                 tc_fence_after();
                 const int vcols = it.valid_cols;
-                const float sc = a.scale_log2e;
-                const uint32_t tbase = tmem + lane_addr + ab * 256 + half * kCols;
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    if (ch * 32 >= vcols) break;
-                    if (wkmax == INT32_MIN || it.cq_max[ch] < wkmin) continue;  // no key of this warp sees the chunk
-                    uint32_t r[32];
-                    tmem_ld32(tbase + ch * 32, r);
+                const uint32_t tbase = tmem + lane_addr + ab * 256 + half * kCols + colh * 64;
+                const int ch0 = colh * 2, ch1 = ch0 + 1;
+                // a chunk is skipped when it holds no column or no key of this warp sees any of its columns
+                const bool do0 = ch0 * 32 < vcols && wkmax != INT32_MIN && it.cq_max[ch0] >= wkmin;
+                const bool do1 = ch1 * 32 < vcols && wkmax != INT32_MIN && it.cq_max[ch1] >= wkmin;
+                uint32_t r[32];
+                if (do0) {
+                    tmem_ld32(tbase, r);
                     tmem_ld_wait();
-                    const float4 *L4 = reinterpret_cast<const float4 *>(it.L + ch * 32);
-                    if ((ch + 1) * 32 <= vcols && it.cq_min[ch] >= wkmax) {
-#pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
-                            const float4 l = L4[c4];
-                            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x));
-                            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y));
-                            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z));
-                            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w));
-                        }
+                    const bool fast = (ch0 + 1) * 32 <= vcols && it.cq_min[ch0] >= wkmax;
+                    epi_chunk(r, it.L + ch0 * 32, it.qp + ch0 * 32, kpos, sc, fast, acc0, acc1);
+                }
+                if (do1) {
+                    tmem_ld32(tbase + 32, r);
+                    tmem_ld_wait();
+                    const bool fast = (ch1 + 1) * 32 <= vcols && it.cq_min[ch1] >= wkmax;
+                    epi_chunk(r, it.L + ch1 * 32, it.qp + ch1 * 32, kpos, sc, fast, acc0, acc1);
+                }
+                tc_fence_before();
+                if (flags & kLast) {
+                    // add the column halves (before the accumulator is released, see below)
+                    const uint32_t p = tcount & 1, ph = (tcount >> 1) & 1;
+                    ++tcount;
+                    if (colh == 1) {
+                        ctl.part[p][key] = acc0 + acc1;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl.part_full[p]);
                     } else {
-                        const int4 *P4 = reinterpret_cast<const int4 *>(it.qp + ch * 32);
-#pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
-                            const float4 l = L4[c4];
-                            const int4 p = P4[c4];
-                            const float x0 = fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x);
-                            const float x1 = fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y);
-                            const float x2 = fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z);
-                            const float x3 = fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w);
-                            acc0 += ex2(p.x >= kpos ? x0 : -INFINITY);
-                            acc1 += ex2(p.y >= kpos ? x1 : -INFINITY);
-                            acc0 += ex2(p.z >= kpos ? x2 : -INFINITY);
-                            acc1 += ex2(p.w >= kpos ? x3 : -INFINITY);
+                        if (!mbar_wait(&ctl.part_full[p], ph, ctl, a.status, row)) break;
+                        if (kv) {
+                            const float v = (acc0 + acc1) + ctl.part[p][key];
+                            *dst = a.accumulate ? *dst + v : v;
                         }
                     }
                 }
-                tc_fence_before();
+                // Releasing the buffer after the column-half exchange keeps part[p] from being rewritten
+                // before it is read: its next writer must first obtain an accumulator this warp released.
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.acc_empty[ab]);
                 if (++ab == 2) { ab = 0; abph ^= 1; }
-            }
-            if (flags & kLast) {
-                if (kv) {
-                    float *dst = a.scores + (int64_t)row * c.max_slots + (int64_t)it.tile * kTileKeys + key;
-                    const float v = acc0 + acc1;
-                    *dst = a.accumulate ? *dst + v : v;
-                }
+            } else if ((flags & kLast) && colh == 0 && kv) {
+                if (!a.accumulate) *dst = 0.f;  // no query sees this tile
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl.m_empty[mk]);

@@ -73,52 +73,73 @@ def algorithmic_work(spec, layout, queries):
 
 
 class ClockSampler:
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = None
+    """SM clock and clock-event reasons sampled through NVML (the source nvidia-smi reads) every 2 ms in a
+    thread while the timed region runs (nvidia-smi's own loop is too coarse for a region this short)."""
+
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap")]
+
+    def __init__(self, torch_index):
+        self.torch_index = torch_index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+        self._thread = None
+        self.err = None
+
+    def _handle(self, nv):
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.torch_index).uuid)
+        except Exception:
+            pass
+        n = nv.nvmlDeviceGetCount()
+        for i in range(n):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            u = nv.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if uuid and u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                return h
+        vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip().isdigit()]
+        return nv.nvmlDeviceGetHandleByIndex(int(vis[self.torch_index]) if self.torch_index < len(vis) else self.torch_index)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report no clocks rather than guess
+            self.err = repr(e)
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for name, attr in self.REASONS:
+                        if bits & getattr(nv, attr):
+                            self.reasons.add(name)
+                except Exception as e:
+                    self.err = repr(e)
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                p = [x.strip() for x in line.split(",")]
-                if len(p) < 9:
-                    continue
-                try:
-                    sm.append(float(p[1]))
-                    mx.append(float(p[2]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, p[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self._thread is None:
+            return {"error": self.err} if self.err else None
+        self._stop.set()
+        self._thread.join()
+        if not self.samples:
+            return {"error": self.err or "no samples"}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "NVML every 2 ms during the timed steps"}
 
 
 def build_workload(device):
@@ -158,24 +179,22 @@ def run_ours(args, rank, world, device):
         rnd.reset_ratchet()
         flush.fill_(1.0)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-
     def step(e=None):
         if e is not None:
-            e[0].record(stream)
+            e[0].record()
         kvc.kvc_confidence_ratchet(logits, rnd.state, rnd.budget, rnd.params, None, rnd.status)
         if e is not None:
-            e[1].record(stream)
+            e[1].record()
         kvc.kvc_score_from_lse(cache, queries, rnd.scores, 0, rnd.status)
         if e is not None:
-            e[2].record(stream)
+            e[2].record()
         kvc.kvc_lrfu_update(cache, rnd.scores, rnd.crf, 0.5, 0.9, 1, 0, rnd.status)
         kvc.kvc_select_budget(cache, rnd.crf, rnd.budget, rnd.keep, rnd.kept, 0, rnd.status)
         kvc.kvc_plan_slots(cache, rnd.keep, rnd.kept, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.status)
         kvc.kvc_compact_pages(cache, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.kept, rnd.crf, rnd.freed,
                               rnd.num_freed, rnd.workspace, rnd.status)
         if e is not None:
-            e[3].record(stream)
+            e[3].record()
 
     for _ in range(args.warmup):
         restore()
@@ -185,24 +204,46 @@ def run_ours(args, rank, world, device):
     if code != 0:
         raise RuntimeError(f"device status {rnd.device_status()} during warm-up")
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    local = torch.cuda.current_device()
-    ids = [x for x in vis.split(",") if x.strip().isdigit()]
-    clocks = ClockSampler(int(ids[local]) if local < len(ids) else local)
+    # the round as one CUDA graph (the six calls, eight kernels), with timing events captured as nodes
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    graph = None
+    if not args.no_graph:
+        restore()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(ev)
+        for _ in range(2):      # replay warm-up
+            restore()
+            graph.replay()
+        torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    step_ms, score_ms, ratchet_ms = [], [], []
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    clocks = ClockSampler(torch.cuda.current_device())
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks.start()
     for k in range(args.steps):
         restore()
-        step(ev[k])
+        if graph is not None:
+            graph.replay()
+            ev[3].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            score_ms.append(ev[1].elapsed_time(ev[2]))
+            ratchet_ms.append(ev[0].elapsed_time(ev[1]))
+        else:
+            step(evs[k])
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    step_ms = [ev[k][0].elapsed_time(ev[k][3]) for k in range(args.steps)]
-    score_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
-    ratchet_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
+    if graph is None:
+        step_ms = [evs[k][0].elapsed_time(evs[k][3]) for k in range(args.steps)]
+        score_ms = [evs[k][1].elapsed_time(evs[k][2]) for k in range(args.steps)]
+        ratchet_ms = [evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)]
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], device=device)
@@ -244,6 +285,7 @@ def run_ours(args, rank, world, device):
         "breakdown_ms": {"ratchet": float(np.mean(ratchet_ms)), "score": score_avg,
                          "lrfu+select+plan+compact": float(np.mean(step_ms) - np.mean(score_ms) - np.mean(ratchet_ms))},
         "gpu_launches": EvictionRound_KERNELS * args.steps,
+        "launch": "CUDA graph of the round" if graph is not None else "direct C-ABI calls",
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clk,
@@ -397,10 +439,11 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

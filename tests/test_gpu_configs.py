@@ -160,18 +160,20 @@ def test_batch16_full_sampled():
 
 def test_streaming_rounds():
     """Streaming shape: beacon + recent queries (LSE computed by the library), 28 q / 4 KV heads, the LRFU state
-    carried across rounds, 64 decoded tokens appended between compactions."""
+    carried across rounds, 64 decoded tokens appended between compactions.  The oracle keeps its own state from
+    the initial generated cache onward; the appended tokens go to pages no block table references (the same
+    pages on both sides)."""
     spec = synth.streaming(num_seqs=2, ctx=2048)
     spec.spare_frac = 0.7
     spec.budget = 1800
     w = H.build(spec)
-    geo, P = w.geo, spec.page_size
+    geo, P, D = w.geo, spec.page_size, spec.head_dim
     rnd = EvictionRound(w.cache)
     rnd.budget.fill_(spec.budget)
-    used = int(sum(-(-int(n) // P) for n in w.layout.row_len.tolist()))
-    next_page = used
-    st = snapshot(w)
-    crf_o = np.zeros((spec.rows, spec.max_slots))
+    o = snapshot(w)                      # oracle state: the generated cache, before any kernel ran
+    o["crf"] = np.zeros((spec.rows, spec.max_slots))
+    in_use = set(int(x) for x in o["bt"][o["bt"] >= 0])
+    free = [p for p in range(w.layout.num_pages) if p not in in_use]
     n_total = [2048] * spec.num_seqs
     for rd in range(10):
         qs = synth.streaming_queries(spec, n_total, device=DEV)
@@ -182,60 +184,60 @@ def test_streaming_rounds():
         assert rnd.device_status()[0] == 0
         hq = qs.q.cpu().to(torch.float64).numpy()
         qpos, numq = qs.q_pos.cpu().numpy(), qs.num_q.cpu().numpy()
-        lse_o = ocache.lse_cache(geo, st["kf"], st["bt"], st["rl"], st["sp"], hq, qpos, numq, qs.max_q)
-        # the library's LSE pass against the oracle's
+        kf = torch.from_numpy(o["k"]).view(torch.bfloat16).to(torch.float64).numpy()
+        lse_o = ocache.lse_cache(geo, kf, o["bt"], o["rl"], o["sp"], hq, qpos, numq, qs.max_q)
         glse = q.lse.cpu().numpy().astype(np.float64)
-        assert np.max(np.abs(glse - lse_o)) < 5e-5
-        osc = ocache.score_cache(geo, st["kf"], st["bt"], st["rl"], st["sp"], hq, lse_o.astype(np.float32),
-                                 qpos, numq)
-        crf_o, ohits = ocache.lrfu_cache(geo, osc, crf_o, st["rl"], st["sp"], 0.5, HIT)
-        okeep, _ = ocache.select_cache(geo, crf_o, st["rl"], st["sp"], st["sl"], [spec.budget] * spec.num_seqs)
+        assert np.max(np.abs(glse - lse_o)) < 5e-5, "the library's LSE pass against the oracle's"
+        osc = ocache.score_cache(geo, kf, o["bt"], o["rl"], o["sp"], hq, lse_o.astype(np.float32), qpos, numq)
+        crf_o, ohits = ocache.lrfu_cache(geo, osc, o["crf"], o["rl"], o["sp"], 0.5, HIT)
+        okeep, _ = ocache.select_cache(geo, crf_o, o["rl"], o["sp"], o["sl"], [spec.budget] * spec.num_seqs)
         gsc, gkeep = rnd.scores.cpu().numpy(), rnd.keep.cpu().numpy()
         same = True
         for r in range(spec.rows):
-            n = int(st["rl"][r])
+            n = int(o["rl"][r])
             H.assert_scores_close(gsc[r, :n], osc[r, :n], f"round {rd} row {r}")
             same &= check_keep(gkeep[r, :n], okeep[r, :n], crf_o[r, :n], osc[r, :n], ohits[r, :n], spec.budget)
         if not same:
             return   # both sides are right; their states part here
-        plans = ocache.plan_cache(geo, okeep, st["rl"])
-        k2, v2, bt2, rl2, sp2, sl2, crf_o, fr = ocache.compact_cache(geo, st["k"], st["v"], st["bt"], st["rl"],
-                                                                     st["sp"], st["sl"], crf_o, plans)
+        plans = ocache.plan_cache(geo, okeep, o["rl"])
+        k2, v2, bt2, rl2, sp2, sl2, crf2, fr = ocache.compact_cache(geo, o["k"], o["v"], o["bt"], o["rl"], o["sp"],
+                                                                    o["sl"], crf_o, plans)
         st1 = snapshot(w)
         for key, val in (("k", k2), ("v", v2), ("bt", bt2), ("rl", rl2), ("sp", sp2), ("sl", sl2)):
             assert np.array_equal(st1[key], val), f"round {rd}: {key}"
         gcrf = rnd.crf.cpu().numpy()
         for r in range(spec.rows):
             m = int(rl2[r])
-            np.testing.assert_allclose(gcrf[r, :m], crf_o[r, :m], rtol=2e-5, atol=1e-30)
-        # append 64 decoded tokens per row (pages from the spare region, same on both sides)
-        bt, rl, sp, sl = bt2.copy(), rl2.copy(), sp2.copy(), sl2.copy()
-        kb, vb = w.cache.k_pool, w.cache.v_pool
+            np.testing.assert_allclose(gcrf[r, :m], crf2[r, :m], rtol=2e-5, atol=1e-30)
+        assert int(rnd.num_freed[0]) == len(fr)
+        free.extend(int(x) for x in fr)
+        # append 64 decoded tokens per row, to both states
+        o = dict(k=k2, v=v2, bt=bt2, rl=rl2, sp=sp2, sl=sl2, crf=crf2)
         for r in range(spec.rows):
             s, l, h = geo.coords(r)
-            m = int(rl[r])
+            m = int(o["rl"][r])
             pos = torch.arange(n_total[s], n_total[s] + 64)
-            for i in range(64):
-                slot = m + i
-                if bt[r, slot // P] < 0:
-                    bt[r, slot // P] = next_page
-                    next_page += 1
+            for slot in range(m, m + 64):
+                if o["bt"][r, slot // P] < 0:
+                    o["bt"][r, slot // P] = free.pop(0)
             slots = np.arange(m, m + 64)
-            phys = torch.from_numpy(bt[r, slots // P].astype(np.int64) * P + slots % P)
-            kb.view(-1, spec.head_dim)[phys.to(DEV)] = synth.key_values(spec, s, l, h, pos.to(DEV), "k")
-            vb.view(-1, spec.head_dim)[phys.to(DEV)] = synth.key_values(spec, s, l, h, pos.to(DEV), "v")
-            sp[r, m:m + 64] = pos.numpy()
-            sl[r, m:m + 64] = synth.LABEL_REASON
-            rl[r] = m + 64
-            crf_o[r, m:m + 64] = 0.0
+            phys = o["bt"][r, slots // P].astype(np.int64) * P + slots % P
+            kv = synth.key_values(spec, s, l, h, pos, "k")
+            vv = synth.key_values(spec, s, l, h, pos, "v")
+            o["k"].reshape(-1, D)[phys] = kv.view(torch.int16).numpy()
+            o["v"].reshape(-1, D)[phys] = vv.view(torch.int16).numpy()
+            w.cache.k_pool.view(-1, D)[torch.from_numpy(phys).to(DEV)] = kv.to(DEV)
+            w.cache.v_pool.view(-1, D)[torch.from_numpy(phys).to(DEV)] = vv.to(DEV)
+            o["sp"][r, m:m + 64] = pos.numpy()
+            o["sl"][r, m:m + 64] = synth.LABEL_REASON
+            o["rl"][r] = m + 64
+            o["crf"][r, m:m + 64] = 0.0
             rnd.crf[r, m:m + 64] = 0.0
-        assert next_page <= w.layout.num_pages
-        w.cache.block_table.copy_(torch.from_numpy(bt))
-        w.cache.row_len.copy_(torch.from_numpy(rl))
-        w.cache.slot_pos.copy_(torch.from_numpy(sp))
-        w.cache.slot_label.copy_(torch.from_numpy(sl))
+        w.cache.block_table.copy_(torch.from_numpy(o["bt"]))
+        w.cache.row_len.copy_(torch.from_numpy(o["rl"]))
+        w.cache.slot_pos.copy_(torch.from_numpy(o["sp"]))
+        w.cache.slot_label.copy_(torch.from_numpy(o["sl"]))
         n_total = [n + 64 for n in n_total]
-        st = snapshot(w)
 
 
 def _stress_cache(S, L, ctx, seed, device=DEV):
