@@ -101,6 +101,15 @@ kvc_status check_params(const kvc_ratchet_params *p) {
 
 }  // namespace
 
+namespace kvc {
+void set_last_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+}  // namespace kvc
+
 extern "C" {
 
 const char *kvc_status_string(kvc_status s) {

@@ -55,4 +55,7 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
 
 size_t ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params &p);
 
+// Sets the thread-local message returned by kvc_last_error().
+void set_last_error(const char *fmt, ...);
+
 }  // namespace kvc

@@ -27,7 +27,8 @@ DEV_CODES = {0: "ok", 1: "bad page", 2: "bad length", 3: "non-finite value", 4: 
 
 EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse", "kvc_score_from_lse",
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
-           "kvc_compact_pages", "kvc_ratchet_state_bytes", "kvc_ratchet_init", "kvc_confidence_ratchet"]
+           "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
+           "kvc_confidence_ratchet"]
 
 
 class KvcCache(ctypes.Structure):
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
             "kvc_plan_slots": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, vp]),
             "kvc_compact_workspace_bytes": (ctypes.c_size_t, [i32]),
             "kvc_compact_pages": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, i64, vp, vp, ctypes.c_size_t, vp, vp]),
+            "kvc_compact_pages_noalloc": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp]),
             "kvc_ratchet_state_bytes": (ctypes.c_size_t, [i32, pr]),
             "kvc_ratchet_init": (ctypes.c_int, [vp, vp, i32, pr, vp]),
             "kvc_confidence_ratchet": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, pr, vp, vp]),
@@ -211,6 +213,21 @@ def kvc_compact_pages(cache: Cache, move_src, move_dst, num_moves, new_len, crf:
                                    _ptr(crf), _ptr(freed), freed.numel(), _ptr(num_freed), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _ptr(d_status), _stream(stream)),
            "kvc_compact_pages")
+
+
+def kvc_compact_pages_noalloc(cache: Cache, move_src, move_dst, num_moves, new_len, crf: Optional[torch.Tensor],
+                              freed: torch.Tensor, num_freed: torch.Tensor, d_status=None, stream=None):
+    """kvc_compact_pages with the library's built-in workspace, for callers that cannot allocate device memory
+    (e.g. during CUDA graph capture, or when the KV pool owns all free memory).  At most KVC_NOALLOC_MAX_ROWS
+    rows; calls that overlap on the GPU share the workspace and must be serialised."""
+    cs = cache.struct()
+    _check(lib().kvc_compact_pages_noalloc(ctypes.byref(cs), _ptr(move_src), _ptr(move_dst), _ptr(num_moves),
+                                           _ptr(new_len), _ptr(crf), _ptr(freed), freed.numel(), _ptr(num_freed),
+                                           _ptr(d_status), _stream(stream)),
+           "kvc_compact_pages_noalloc")
+
+
+NOALLOC_MAX_ROWS = 16384
 
 
 def kvc_ratchet_state_bytes(num_seqs: int, params: KvcRatchetParams) -> int:

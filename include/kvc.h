@@ -244,6 +244,25 @@ kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, co
                              void *workspace, size_t workspace_bytes, int32_t *d_status,
                              kvc_stream_t stream);
 
+/*
+ * kvc_compact_pages without a caller-provided workspace, for callers that cannot allocate
+ * device memory: code running during CUDA graph capture (an allocation there breaks the
+ * capture), engines whose allocator has given all free memory to the KV pool, or
+ * foreign-function callers with no access to the host framework's allocator.  The pages
+ * describe no such variant; it exists for those callers only.
+ * Same arguments, checks and results as kvc_compact_pages, minus workspace/workspace_bytes:
+ * the workspace is a fixed array inside the library (KVC_NOALLOC_MAX_ROWS + 1 int64 per
+ * GPU, held from library load to process exit).  Calls for more than KVC_NOALLOC_MAX_ROWS
+ * rows return KVC_ERR_UNSUPPORTED.  The first call on each device looks up the array's
+ * device address (make it before any stream capture).  All calls share the array, so calls
+ * whose kernels can overlap on the GPU race and must be serialised by the caller.
+ */
+#define KVC_NOALLOC_MAX_ROWS 16384
+kvc_status kvc_compact_pages_noalloc(const kvc_cache *cache, const int32_t *move_src, const int32_t *move_dst,
+                                     const int32_t *num_moves, const int32_t *new_len, float *crf,
+                                     int32_t *freed, int64_t freed_capacity, int64_t *num_freed,
+                                     int32_t *d_status, kvc_stream_t stream);
+
 /* bytes of the ratchet state buffer for num_seqs sequences */
 size_t kvc_ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params *params);
 
