@@ -51,11 +51,22 @@ __global__ void __launch_bounds__(kThreads) lrfu_kernel(LrfuArgs a) {
     // stage the slice (raw fp32 bits, sign cleared so -0.0 ranks as 0), validate, row maximum
     int bad = 0;
     float mx = 0.f;
-    for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-        const float v = s[i];
-        if (!is_finite(v) || v < 0.f) bad = 1;
-        mx = fmaxf(mx, v);
-        if (cached) kc[i - lo] = __float_as_uint(v) & 0x7fffffffu;
+    for (int base = lo + threadIdx.x; base < hi; base += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {  // eight independent loads in flight before any is used
+            const int i = base + u * blockDim.x;
+            v[u] = i < hi ? s[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < hi) {
+                if (!is_finite(v[u]) || v[u] < 0.f) bad = 1;
+                mx = fmaxf(mx, v[u]);
+                if (cached) kc[i - lo] = __float_as_uint(v[u]) & 0x7fffffffu;
+            }
+        }
     }
     row_max_or(rc, sh, mx, bad);
     if (bad) {
@@ -124,9 +135,21 @@ __global__ void __launch_bounds__(kThreads) lrfu_kernel(LrfuArgs a) {
         row_ordered_ranks(rc, sh, lo, hi, [&](int i) { return is_hit(i) < 0; },
                           [&](int i, int rank) { update(i, (unsigned long long)rank < slot_need); });
     }
-    for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-        const int hit = is_hit(i);
-        if (hit >= 0) update(i, hit);
+    for (int base = lo + threadIdx.x; base < hi; base += 8 * blockDim.x) {
+        float old[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * blockDim.x;
+            old[u] = i < hi ? crf[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < hi) {
+                const int hit = is_hit(i);
+                if (hit >= 0) crf[i] = fmaf(a.decay, old[u], hit ? (a.binary ? 1.f : sval(i)) : 0.f);
+            }
+        }
     }
     rc.cl.sync();  // peers may still read this CTA's shared memory
 }

@@ -10,10 +10,12 @@
 // Launch A (confidence): a cluster of kCluster CTAs per (sequence, step) row of
 //   logits.  Each CTA stages its slice of the vocabulary in shared memory, reduces
 //   its (max, sum of exp) and its exact top-k list, and the leader CTA merges the
-//   cluster's partials through distributed shared memory into c_t.  The local top-k
-//   uses the k-th largest of the per-thread maxima as a lower bound to pick a short
-//   candidate list; when that list overflows (many equal logits) it falls back to an
-//   exact radix search over the staged slice.
+//   cluster's partials through distributed shared memory into c_t.  The slice arrives
+//   by bulk (TMA) copies when the row is 16-byte aligned.  The local top-k takes the
+//   k-th largest of the warps' top-2 per-thread maxima as a lower bound, collects the
+//   values above it (a few dozen) and sorts them with a warp bitonic network; when
+//   more than 64 qualify (many equal logits) it falls back to an exact radix search
+//   over the staged slice.
 // Launch B (ratchet): one warp per sequence pools the newly completed windows,
 //   updates the least-squares sums, evaluates the fit once and moves the budget.
 #include <cooperative_groups.h>
@@ -50,38 +52,49 @@ struct ConfArgs {
     const float *logits;
     int32_t steps, vocab, chunk;
     int32_t top_k;
+    int32_t bulk;       // rows and slices 16-byte aligned: stage with bulk copies
     float *hist;        // [seqs][hist_len]
     int32_t hist_len, window;
     float *conf_out;    // [seqs][steps] or null
     int32_t *status;
 };
 
-// Descending bitonic sort of kThreads floats in shared memory (all threads take part).
-__device__ void bitonic_desc(float *v) {
-    const int i = threadIdx.x;
-    for (int k = 2; k <= kThreads; k <<= 1) {
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Descending sort of 64 values held two per lane (lane l holds v[0] = x[l], v[1] = x[l + 32]) with a
+// bitonic network over the warp.
+__device__ __forceinline__ void warp_sort64_desc(float &a, float &b) {
+    const int lane = threadIdx.x & 31;
+    // element index e = lane (a) and lane + 32 (b)
+    for (int k = 2; k <= 64; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
-            const int ixj = i ^ j;
-            if (ixj > i) {
-                const float a = v[i], b = v[ixj];
-                const bool desc = (i & k) == 0;
-                if (desc ? (a < b) : (a > b)) {
-                    v[i] = b;
-                    v[ixj] = a;
-                }
+            if (j == 32) {
+                // partners are a and b of the same lane
+                const bool desc = (lane & k) == 0;  // k == 64 here: whole array descending
+                const float hi = fmaxf(a, b), lo = fminf(a, b);
+                a = desc ? hi : lo;
+                b = desc ? lo : hi;
+            } else {
+                const float pa = __shfl_xor_sync(0xffffffffu, a, j);
+                const float pb = __shfl_xor_sync(0xffffffffu, b, j);
+                const bool lower = (lane & j) == 0;
+                const bool da = (lane & k) == 0, db = ((lane + 32) & k) == 0;
+                a = (lower == da) ? fmaxf(a, pa) : fminf(a, pa);
+                b = (lower == db) ? fmaxf(b, pb) : fminf(b, pb);
             }
-            __syncthreads();
         }
     }
 }
 
 struct ConfShared {
     RadixShared rs;
-    float sortbuf[kThreads];
+    float cand[64];
     float topk[kMaxTopK];
+    float wtop[32];      // top-2 per warp of the per-thread maxima
     float red_f[32];
     double red_d[32];
     int red_i[32];
+    uint64_t bar;
     float cmax;
     double csum;
     int ncand;
@@ -98,57 +111,116 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
     const float *row = a.logits + ((int64_t)seq * a.steps + step) * a.vocab;
     const int lo = min(a.vocab, rank * a.chunk), hi = min(a.vocab, lo + a.chunk);
     const int cnt = hi - lo;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // stage the slice, per-thread maximum, finiteness
+    // stage the slice in shared memory: one bulk copy when the row slice is 16-byte aligned
+    if (tid == 0) {
+        sh.ncand = 0;
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&sh.bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const bool bulk = a.bulk && cnt > 0;
+    if (bulk) {
+        if (tid == 0) {
+            const uint32_t bytes = (uint32_t)cnt * 4u;
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&sh.bar)), "r"(bytes)
+                         : "memory");
+            for (uint32_t off = 0; off < bytes; off += 16384u) {
+                const uint32_t sz = min(16384u, bytes - off);
+                asm volatile(
+                    "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                        smem_addr(zs) + off),
+                    "l"(reinterpret_cast<const char *>(row + lo) + off), "r"(sz), "r"(smem_addr(&sh.bar))
+                    : "memory");
+            }
+        }
+        // bounded wait for the copy (a second at most)
+        uint32_t done = 0;
+        long long t0 = clock64();
+        while (!done) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+                : "=r"(done)
+                : "r"(smem_addr(&sh.bar))
+                : "memory");
+            if (!done && clock64() - t0 > (1ll << 31)) {
+                if (tid == 0) report(a.status, KVC_DEV_TIMEOUT, seq);
+                break;
+            }
+        }
+    } else {
+        for (int i = tid; i < cnt; i += kThreads) zs[i] = row[lo + i];
+        __syncthreads();
+    }
+    // per-thread maximum and finiteness (from shared memory)
     float tmax = -INFINITY;
     int bad = 0;
     for (int i = tid; i < cnt; i += kThreads) {
-        const float z = row[lo + i];
+        const float z = zs[i];
         bad |= !is_finite(z);
-        zs[i] = z;
         tmax = fmaxf(tmax, z);
     }
-    if (tid == 0) sh.ncand = 0;
-    const float cmax = block_max(tmax, sh.red_f);
-    bad = block_or(bad, sh.red_i);
-    float part = 0.f;
-    if (cmax != -INFINITY)
-        for (int i = tid; i < cnt; i += kThreads) part += expf(zs[i] - cmax);
-    const double csum = block_sum<double>((double)part, sh.red_d);
-
-    // lower bound tau0 for the slice's k-th largest: the k-th largest per-thread maximum
-    sh.sortbuf[tid] = tmax;
-    __syncthreads();
-    bitonic_desc(sh.sortbuf);
-    const float tau0 = (cnt >= K) ? sh.sortbuf[K - 1] : -INFINITY;
-    __syncthreads();
-    // candidates z >= tau0
-    sh.sortbuf[tid] = -INFINITY;
-    __syncthreads();
-    for (int i = tid; i < cnt; i += kThreads) {
-        const float z = zs[i];
-        if (z >= tau0) {
-            const int at = atomicAdd(&sh.ncand, 1);
-            if (at < kThreads) sh.sortbuf[at] = z;
+    // lower bound tau0 for the slice's k-th largest: the k-th largest of the 32 warp top-2 values
+    {
+        float m1 = tmax;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        const unsigned who = __ballot_sync(0xffffffffu, tmax == m1);
+        float m2 = (lane == __ffs(who) - 1) ? -INFINITY : tmax;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+        if (lane == 0) {
+            sh.wtop[2 * warp] = m1;
+            sh.wtop[2 * warp + 1] = m2;
         }
     }
-    __syncthreads();
+    const float cmax = block_max(tmax, sh.red_f);   // also orders the wtop writes
+    bad = block_or(bad, sh.red_i);
+    float tau0 = -INFINITY;
+    if (cnt >= K && K <= 2 * (kThreads / 32)) {
+        // every thread ranks the 32 candidates for the bound; identical in all threads
+        const float v = sh.wtop[lane];
+        int above = 0;
+        for (int f = 0; f < 32; ++f) {
+            const float w = sh.wtop[f];
+            above += (w > v) || (w == v && f < lane);
+        }
+        const unsigned is_k = __ballot_sync(0xffffffffu, above == K - 1);
+        tau0 = __shfl_sync(0xffffffffu, v, __ffs(is_k) - 1);
+    }
+    // log-sum-exp partial and candidates z >= tau0 (one pass over shared memory)
+    float part = 0.f;
+    if (cmax != -INFINITY) {
+        for (int i = tid; i < cnt; i += kThreads) {
+            const float z = zs[i];
+            part += expf(z - cmax);
+            if (z >= tau0) {
+                const int at = atomicAdd(&sh.ncand, 1);
+                if (at < 64) sh.cand[at] = z;
+            }
+        }
+    }
+    const double csum = block_sum<double>((double)part, sh.red_d);  // also orders the candidate writes
     const int ncand = sh.ncand;
-    if (ncand <= kThreads) {
-        bitonic_desc(sh.sortbuf);
-        if (tid < K) sh.topk[tid] = sh.sortbuf[tid];  // -inf pads a slice shorter than k
+    if (ncand <= 64) {
+        if (warp == 0) {
+            float x = lane < ncand ? sh.cand[lane] : -INFINITY;
+            float y = lane + 32 < ncand ? sh.cand[lane + 32] : -INFINITY;
+            warp_sort64_desc(x, y);
+            if (lane < K) sh.topk[lane] = x;  // -inf pads a slice shorter than k
+            if (lane + 32 < K) sh.topk[lane + 32] = y;
+        }
     } else {
-        // exact fallback: k-th largest key over the staged slice, then values above it
-        RadixResult r = radix_search_desc<false>(
+        // exact fallback (many equal logits): k-th largest key over the staged slice, then values above it
+        const RadixResult r = radix_search_desc<false>(
             cnt, (unsigned long long)K, [&](int i) { return float_key(zs[i]); }, [](int) { return 1ull; },
             [](int) { return true; }, sh.rs);
         const float T = key_float(r.key);
         if (tid == 0) sh.ncand = 0;
         __syncthreads();
-        for (int i = tid; i < cnt; i += kThreads) {
+        for (int i = tid; i < cnt; i += kThreads)
             if (float_key(zs[i]) > r.key) sh.topk[atomicAdd(&sh.ncand, 1)] = zs[i];
-        }
         __syncthreads();
         for (int t = (int)r.above + tid; t < K; t += kThreads) sh.topk[t] = T;
     }
@@ -317,11 +389,12 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
     auto *st = static_cast<kvc_ratchet_seq_state *>(state);
     float *hist = reinterpret_cast<float *>(static_cast<char *>(state) + l.state_bytes);
     if (steps > 0) {
-        const int chunk = (vocab + kCluster - 1) / kCluster;
+        const int chunk = ((vocab + kCluster - 1) / kCluster + 3) / 4 * 4;  // whole 16-byte units per slice
         const size_t smem = (size_t)chunk * sizeof(float);
         cudaError_t e = cudaFuncSetAttribute(confidence_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        ConfArgs a{logits, steps, vocab, chunk, p.top_k, hist, l.hist_len, p.window, conf_out, status};
+        const int bulk = (vocab % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
+        ConfArgs a{logits, steps, vocab, chunk, p.top_k, bulk, hist, l.hist_len, p.window, conf_out, status};
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(kCluster, (unsigned)steps, (unsigned)num_seqs);
         cfg.blockDim = dim3(kThreads);

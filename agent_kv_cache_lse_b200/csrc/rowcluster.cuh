@@ -28,7 +28,6 @@ struct RowHist {
 
 struct RowShared {
     RowHist hist[2];
-    unsigned long long lane_w[32][32];  // per warp, per lane: weights combined by a group leader
     unsigned int gcnt[kRowBins];        // cluster-wide histogram of the current pass
     unsigned long long gwt[kRowBins];
     // published scalars, double-buffered
@@ -140,7 +139,7 @@ __device__ inline unsigned long long row_sum_u64(RowCtx &rc, RowShared &sh, unsi
 template <bool kMass, typename KeyFn, typename WeightFn, typename ValidFn>
 __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi, unsigned long long target,
                                       KeyFn key, WeightFn weight, ValidFn valid) {
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) {
         sh.prefix = 0;
         sh.pmask = 0;
@@ -172,40 +171,37 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
                 if (kMass && in) wv = weight(i);
             }
             const unsigned active = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const uint32_t bin = (k >> shift) & (kRowBins - 1);
-                const unsigned peers = __match_any_sync(active, bin);
-                const int leader = __ffs(peers) - 1;
-                if (kMass) sh.lane_w[wid][lane] = wv;
-                __syncwarp(active);
-                if (lane == leader) {
-                    atomicAdd(&h.cnt[bin], (unsigned)__popc(peers));
-                    if (kMass) {
-                        unsigned long long s = 0;
-                        if (peers == 0xffffffffu) {
-                            // whole warp in one bin: tree-free sum in registers of the leader
-                            for (int l = 0; l < 32; ++l) s += sh.lane_w[wid][l];
-                        } else {
-                            unsigned p = peers;
-                            while (p) {
-                                s += sh.lane_w[wid][__ffs(p) - 1];
-                                p &= p - 1;
-                            }
-                        }
-                        atomicAdd(&h.wt[bin], s);
-                    }
+            if (active == 0u) continue;
+            // a warp whose taking part lanes all share one digit (the common case: rows full of equal or
+            // similar values) adds with one atomic; otherwise every lane adds its own
+            const uint32_t bin = (k >> shift) & (kRowBins - 1);
+            const int first = __ffs(active) - 1;
+            const uint32_t bin0 = __shfl_sync(0xffffffffu, bin, first);
+            const bool uniform = __all_sync(0xffffffffu, !in || bin == bin0);
+            if (uniform) {
+                if (kMass) {
+                    unsigned long long s = wv;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                    if (lane == first) atomicAdd(&h.wt[bin0], s);
                 }
-                __syncwarp(active);
+                if (lane == first) atomicAdd(&h.cnt[bin0], (unsigned)__popc(active));
+            } else if (in) {
+                atomicAdd(&h.cnt[bin], 1u);
+                if (kMass) atomicAdd(&h.wt[bin], wv);
             }
         }
         rc.cl.sync();
         for (int i = tid; i < kRowBins; i += blockDim.x) {
             unsigned int c = 0;
             unsigned long long w = 0;
-            for (int r = 0; r < rc.nranks; ++r) {
-                const RowHist &rh = rc.cl.map_shared_rank(&sh, r)->hist[b];
-                c += rh.cnt[i];
-                if (kMass) w += rh.wt[i];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {  // all remote reads issued before the sums need them
+                if (r < rc.nranks) {
+                    const RowHist &rh = rc.cl.map_shared_rank(&sh, r)->hist[b];
+                    c += rh.cnt[i];
+                    if (kMass) w += rh.wt[i];
+                }
             }
             sh.gcnt[i] = c;
             sh.gwt[i] = kMass ? w : (unsigned long long)c;

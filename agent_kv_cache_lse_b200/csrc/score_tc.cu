@@ -61,6 +61,12 @@ struct alignas(16) Item {
 static_assert(sizeof(Item) % 16 == 0, "items hold float4-read arrays");
 constexpr int kFirst = 1, kLast = 2;
 
+struct TileInfo {
+    int row, t, seq, layer, kvh, n_keys, first_vis, last_vis, kmin, nq;
+    unsigned okmask;
+    int page[kPagesPerTile];  // physical page of each of the tile's 16 pages (-1: none or invalid)
+};
+
 struct Ctrl {
     uint64_t q_full[8], q_empty[8];
     uint64_t a_full[2], a_empty[2];        // double-buffered K tile
@@ -72,6 +78,10 @@ struct Ctrl {
     int32_t abort;
     int32_t blk_qmin[kMaxBlocks], blk_qmax[kMaxBlocks];
     float part[2][kTileKeys];
+    int32_t kstage[2][kTileKeys];     // producer: key positions of the current and the next tile
+    uint32_t kvstage[2][8];           // producer: their readable-key masks
+    uint32_t vstage[2][kMaxBlocks / 32];  // producer: their visible-block masks
+    TileInfo tinfo[2];                // producer: decoded current and next tile
 };
 
 struct TcArgs {
@@ -321,19 +331,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_tx_page = 16 * 128;                 // one 16-row, 128-byte box
         const uint32_t q_tx = (uint32_t)(G * nqb) * 128u;    // one Q box per 64-column chunk
         bool ok = true;
-        for (int64_t tid = blockIdx.x; ok && tid < a.total_tiles; tid += gridDim.x) {
+        // ---- tile bookkeeping, prefetched one tile ahead.  Raw loads (row length, the tile's block-table
+        // entries and slot positions, and the first visible block's column data) are issued a whole tile
+        // before they are used, and nothing branches on a loaded value until then.
+        const int mp = c.max_pages_per_row;
+        const int64_t ms = c.max_slots;
+        struct TileRaw {
+            int64_t tid;
+            int n, page, kp[8];
+        };
+        struct ColRaw {
+            float l[4];
+            int p[4];
+        };
+        auto issue_tile = [&](int64_t tid, TileRaw &r) {
+            r.tid = tid;
+            if (tid >= a.total_tiles) return;
             const int64_t rr = tid % RPS, rest = tid / RPS;
             const int t = (int)(rest % a.tiles_per_row), seq = (int)(rest / a.tiles_per_row);
+            const int64_t row = (int64_t)seq * RPS + rr;
+            r.n = c.row_len[row];
+            r.page = c.block_table[row * mp + min(t * kPagesPerTile + (lane & 15), mp - 1)];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                r.kp[i] = c.slot_pos[row * ms + min((int64_t)t * kTileKeys + i * 32 + lane, ms - 1)];
+        };
+        // Decode a tile (waits for its raw loads).  Returns false for a tile with no keys.
+        auto make_info = [&](const TileRaw &r, int parity) -> bool {
+            TileInfo &f = ctl.tinfo[parity];
+            if (r.tid >= a.total_tiles) return false;
+            const int64_t rr = r.tid % RPS, rest = r.tid / RPS;
+            const int t = (int)(rest % a.tiles_per_row);
+            const int seq = (int)(rest / a.tiles_per_row);
             const int row = seq * RPS + (int)rr;
-            const int n = c.row_len[row];
-            if (n < 0 || n > c.max_slots) {
+            const int n = r.n;
+            if (n < 0 || n > ms) {
                 if (t == 0 && lane == 0) report(a.status, KVC_DEV_BAD_LENGTH, row);
-                continue;
+                return false;
             }
             const int k0 = t * kTileKeys;
-            if (k0 >= n) continue;
+            if (k0 >= n) return false;
             const int n_keys = min(kTileKeys, n - k0);
-            const int layer = (int)(rr / c.num_kv_heads), kvh = (int)(rr % c.num_kv_heads);
             if (seq != cur_seq) {
                 cur_seq = seq;
                 nq = min(a.q.num_q[seq], a.q.max_q);
@@ -351,59 +389,124 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-            // pages of the tile (lanes 0..15) and keys' positions (8 per lane)
-            int page = -1;
             bool page_ok = false;
             if (lane < kPagesPerTile && k0 + lane * 16 < n) {
-                page = c.block_table[(int64_t)row * c.max_pages_per_row + t * kPagesPerTile + lane];
-                page_ok = page >= 0 && page < c.num_pages;
+                page_ok = r.page >= 0 && r.page < c.num_pages;
                 if (!page_ok) report(a.status, KVC_DEV_BAD_PAGE, row);
             }
+            if (lane < kPagesPerTile) f.page[lane] = page_ok ? r.page : -1;
             const unsigned okmask = __ballot_sync(0xffffffffu, page_ok);
-            int kp[8];
             int kmin = INT32_MAX;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int key = i * 32 + lane;
                 const bool v = key < n_keys && ((okmask >> (key >> 4)) & 1u);
-                kp[i] = v ? c.slot_pos[(int64_t)row * c.max_slots + k0 + key] : INT32_MAX;
-                if (v) kmin = min(kmin, kp[i]);
+                const int kp = v ? r.kp[i] : INT32_MAX;
+                ctl.kstage[parity][key] = kp;
+                if (v) kmin = min(kmin, kp);
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
             // visible blocks: some query at or after the tile's first key position
             int first_vis = -1, last_vis = -1;
-            for (int b0 = 0; b0 < nblk; b0 += 32) {
+            for (int b0 = 0; b0 < kMaxBlocks; b0 += 32) {
                 const int b = b0 + lane;
                 const bool v = b < nblk && ctl.blk_qmax[b] >= kmin;
                 const unsigned m = __ballot_sync(0xffffffffu, v);
+                if (lane == 0) ctl.vstage[parity][b0 >> 5] = m;
                 if (m) {
                     if (first_vis < 0) first_vis = b0 + __ffs(m) - 1;
                     last_vis = b0 + 31 - __clz(m);
                 }
             }
-            auto fill_tile_part = [&](Item &it, int flags) {
+            if (lane < 8) {
+                uint32_t w = 0;
+                for (int bit = 0; bit < 32; ++bit) {
+                    const int key = lane * 32 + bit;
+                    if (key < n_keys && ((okmask >> (key >> 4)) & 1u)) w |= 1u << bit;
+                }
+                ctl.kvstage[parity][lane] = w;
+            }
+            if (lane == 0) {
+                f.row = row;
+                f.t = t;
+                f.seq = seq;
+                f.layer = (int)(rr / c.num_kv_heads);
+                f.kvh = (int)(rr % c.num_kv_heads);
+                f.n_keys = n_keys;
+                f.first_vis = first_vis;
+                f.last_vis = last_vis;
+                f.kmin = kmin;
+                f.nq = nq;
+                f.okmask = okmask;
+            }
+            __syncwarp();
+            return true;
+        };
+        auto next_visible = [&](int parity, int b) -> int {
+            for (int x = b + 1; x < kMaxBlocks; ++x) {
+                const uint32_t w = ctl.vstage[parity][x >> 5] >> (x & 31);
+                if (w == 0u) {
+                    x = (x | 31);
+                    continue;
+                }
+                return x + __ffs(w) - 1;
+            }
+            return -1;
+        };
+        auto issue_cols = [&](const TileInfo &f, int b, ColRaw &cr) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) it.kpos[i * 32 + lane] = kp[i];
-                if (lane < 8) {
-                    uint32_t w = 0;
-                    for (int bit = 0; bit < 32; ++bit) {
-                        const int key = lane * 32 + bit;
-                        if (key < n_keys && ((okmask >> (key >> 4)) & 1u)) w |= 1u << bit;
-                    }
-                    it.kvalid[lane] = w;
-                }
-                if (lane == 0) {
-                    it.row = row;
-                    it.tile = t;
-                    it.n_keys = n_keys;
-                    it.flags = flags;
-                }
-            };
-            if (first_vis < 0) {
-                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, row)) { ok = false; break; }
+            for (int u = 0; u < 4; ++u) {
+                const int col = u * 32 + lane, jl = col / G, g = col % G;
+                const int j = min(b * nqb + jl, a.q.max_q - 1);
+                cr.l[u] = a.q.lse[((int64_t)(f.seq * c.num_layers + f.layer) * Hq + f.kvh * G + g) * a.q.max_q + j];
+                cr.p[u] = a.q.q_pos[(int64_t)f.seq * a.q.max_q + j];
+            }
+        };
+        auto fill_tile_part = [&](Item &it, const TileInfo &f, int parity, int flags) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) it.kpos[i * 32 + lane] = ctl.kstage[parity][i * 32 + lane];
+            if (lane < 8) it.kvalid[lane] = ctl.kvstage[parity][lane];
+            if (lane == 0) {
+                it.row = f.row;
+                it.tile = f.t;
+                it.n_keys = f.n_keys;
+                it.flags = flags;
+            }
+        };
+
+        TileRaw raw;
+        ColRaw ccur, cnxt;
+        int par = 0;
+        int64_t tid_next = blockIdx.x;
+        // find the first tile with keys
+        bool have = false;
+        while (!have && tid_next < a.total_tiles) {
+            issue_tile(tid_next, raw);
+            tid_next += gridDim.x;
+            have = make_info(raw, par);
+        }
+        if (have && ctl.tinfo[par].first_vis >= 0) issue_cols(ctl.tinfo[par], ctl.tinfo[par].first_vis, cnxt);
+        if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
+        while (ok && have) {
+            ccur = cnxt;
+            const int cpar = par;
+            const TileInfo &cur = ctl.tinfo[cpar];
+            // decode the following tile now (its loads were issued a tile ago) and issue its first columns
+            par ^= 1;
+            have = false;
+            while (!have && tid_next < a.total_tiles) {
+                const TileRaw r = raw;
+                tid_next += gridDim.x;
+                if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
+                have = make_info(r, par);
+            }
+            if (have && ctl.tinfo[par].first_vis >= 0) issue_cols(ctl.tinfo[par], ctl.tinfo[par].first_vis, cnxt);
+
+            if (cur.first_vis < 0) {
+                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
-                fill_tile_part(it, kFirst | kLast);
+                fill_tile_part(it, cur, cpar, kFirst | kLast);
                 if (lane == 0) {
                     it.blk = -1;
                     it.valid_cols = 0;
@@ -415,70 +518,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // K tile into the free buffer: one box per (page, 64-column chunk)
             const uint32_t abuf = ta & 1;
-            if (!mbar_wait(&ctl.a_empty[abuf], ((ta >> 1) & 1) ^ 1, ctl, a.status, row)) { ok = false; break; }
+            if (!mbar_wait(&ctl.a_empty[abuf], ((ta >> 1) & 1) ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
             ++ta;
-            if (lane == 0) mbar_expect_tx(&ctl.a_full[abuf], (uint32_t)__popc(okmask) * a_tx_page * PL::kChunks);
+            if (lane == 0) mbar_expect_tx(&ctl.a_full[abuf], (uint32_t)__popc(cur.okmask) * a_tx_page * PL::kChunks);
             __syncwarp();
-            if (page_ok) {
+            const int my_page = lane < kPagesPerTile ? cur.page[lane] : -1;
+            if (my_page >= 0) {
                 const int half = lane >> 3, r0 = (lane & 7) * 16;
 #pragma unroll
                 for (int kc = 0; kc < PL::kChunks; ++kc) {
                     const uint32_t dst =
                         smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
-                    tma_load_2d(dst, &tmap_k, &ctl.a_full[abuf], kc * 64, page * 16);
+                    tma_load_2d(dst, &tmap_k, &ctl.a_full[abuf], kc * 64, my_page * 16);
                 }
             }
-            // column metadata of a block: 4 columns per lane, prefetched one block ahead
-            auto load_cols = [&](int b, float (&L)[4], int (&P)[4]) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int col = u * 32 + lane, jl = col / G, g = col % G, j = b * nqb + jl;
-                    L[u] = INFINITY;
-                    P[u] = INT32_MIN;
-                    if (jl < nqb && j < nq) {
-                        const float l = a.q.lse[((int64_t)(seq * c.num_layers + layer) * Hq + kvh * G + g) * a.q.max_q + j];
-                        if (l == -INFINITY) {
-                            // a column that saw no key contributes nothing
-                        } else if (!is_finite(l)) {
-                            report(a.status, KVC_DEV_NONFINITE, row);
-                        } else {
-                            L[u] = l * 1.4426950408889634f;
-                            P[u] = a.q.q_pos[(int64_t)seq * a.q.max_q + j];
-                        }
-                    }
-                }
-            };
-            float L[4], Ln[4];
-            int P[4], Pn[4];
-            load_cols(first_vis, L, P);
-            for (int b = first_vis; b >= 0;) {
-                int bn = -1;
-                for (int x = b + 1; x <= last_vis; ++x)
-                    if (ctl.blk_qmax[x] >= kmin) { bn = x; break; }
-                if (bn >= 0) load_cols(bn, Ln, Pn);
+            for (int b = cur.first_vis; b >= 0;) {
+                const int bn = next_visible(cpar, b);
+                ColRaw cn;
+                if (bn >= 0) issue_cols(cur, bn, cn);
                 // Q block b
-                if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_expect_tx(&ctl.q_full[qs], q_tx * PL::kChunks);
 #pragma unroll
                     for (int kc = 0; kc < PL::kChunks; ++kc) {
                         const uint32_t dst = smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128));
-                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, kvh * G, b * nqb, seq * c.num_layers + layer);
+                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, cur.kvh * G, b * nqb,
+                                    cur.seq * c.num_layers + cur.layer);
                     }
                 }
                 if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
-                // metadata item
-                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                // metadata item (the column data was loaded a block earlier)
+                if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
-                const int flags = (b == first_vis ? kFirst : 0) | (b == last_vis ? kLast : 0);
-                if (flags & kFirst) fill_tile_part(it, flags);
-                int vq = min(nqb, nq - b * nqb);
-                const int vcols = vq * G;
+                const int flags = (b == cur.first_vis ? kFirst : 0) | (b == cur.last_vis ? kLast : 0);
+                if (flags & kFirst) fill_tile_part(it, cur, cpar, flags);
+                const int vq = min(nqb, cur.nq - b * nqb);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    it.L[u * 32 + lane] = L[u];
-                    it.qp[u * 32 + lane] = P[u];
-                    int mn = P[u] == INT32_MIN ? INT32_MAX : P[u], mx = P[u];
+                    const int col = u * 32 + lane, jl = col / G;
+                    float Lv = INFINITY;
+                    int Pv = INT32_MIN;
+                    if (jl < vq) {
+                        const float l = ccur.l[u];
+                        if (l == -INFINITY) {
+                            // a column that saw no key contributes nothing
+                        } else if (!is_finite(l)) {
+                            report(a.status, KVC_DEV_NONFINITE, cur.row);
+                        } else {
+                            Lv = l * 1.4426950408889634f;
+                            Pv = ccur.p[u];
+                        }
+                    }
+                    it.L[col] = Lv;
+                    it.qp[col] = Pv;
+                    int mn = Pv == INT32_MIN ? INT32_MAX : Pv, mx = Pv;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -490,22 +584,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (lane == 0) {
-                    it.row = row;
-                    it.tile = t;
+                    it.row = cur.row;
+                    it.tile = cur.t;
                     it.blk = b;
                     it.flags = flags;
-                    it.n_keys = n_keys;
-                    it.valid_cols = vcols;
+                    it.n_keys = cur.n_keys;
+                    it.valid_cols = vq * G;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
                 b = bn;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    L[u] = Ln[u];
-                    P[u] = Pn[u];
-                }
+                ccur = cn;
             }
         }
         // end-of-work marker

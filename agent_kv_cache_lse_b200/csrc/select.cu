@@ -52,11 +52,22 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     auto prot = [&](int i) -> bool { return protect && ((protect >> (lab[i] & 31)) & 1u); };
 
     int bad = 0, nprot = 0;
-    for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-        const float v = crf[i];
-        if (!is_finite(v)) bad = 1;
-        if (cached) kc[i - lo] = float_key(v == 0.f ? 0.f : v);  // -0.0 ranks as +0.0
-        nprot += prot(i) ? 1 : 0;
+    for (int base = lo + threadIdx.x; base < hi; base += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {  // eight independent loads in flight before any is used
+            const int i = base + u * blockDim.x;
+            v[u] = i < hi ? crf[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < hi) {
+                if (!is_finite(v[u])) bad = 1;
+                if (cached) kc[i - lo] = float_key(v[u] == 0.f ? 0.f : v[u]);  // -0.0 ranks as +0.0
+                nprot += prot(i) ? 1 : 0;
+            }
+        }
     }
     float dummy = 0.f;
     row_max_or(rc, sh, dummy, bad);
