@@ -29,7 +29,7 @@ struct LrfuArgs {
     int slice_cap;    // scores cached in shared memory when a CTA's slice fits
 };
 
-__global__ void __launch_bounds__(kThreads) lrfu_kernel(LrfuArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) lrfu_kernel(LrfuArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RowShared &sh = *reinterpret_cast<RowShared *>(smem_raw);
     uint32_t *kc = reinterpret_cast<uint32_t *>(smem_raw + sizeof(RowShared));
@@ -161,7 +161,9 @@ cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, flo
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int C = row_cluster_size(c.rows, sms);
+    int C = row_cluster_size(c.rows, sms);
+    while (C < 8 && (c.max_slots + C - 1) / C > 65536) C <<= 1;  // the mass chunks need slices of at most 2^16
+    if ((c.max_slots + C - 1) / C > 65536) return cudaErrorInvalidValue;
     const int per = (int)((c.max_slots + C - 1) / C);
     const int cap = per < 40960 ? per : 0;
     const size_t smem = sizeof(RowShared) + (size_t)cap * 4;

@@ -21,9 +21,13 @@ namespace cg = cooperative_groups;
 
 constexpr int kRowBins = 256;  // 8-bit digits, 4 passes over 32-bit keys
 
+// Per-CTA histogram of one digit.  A mass is a fixed-point integer below 2^48, kept as three 16-bit
+// chunks summed in 32-bit counters (a CTA's slice holds at most 65,536 entries, so no chunk sum can
+// overflow); the cluster gather recombines them exactly in 64 bits.  Native 32-bit shared-memory atomics
+// stay fast under the heavy contention of rows full of similar values, where 64-bit ones do not.
 struct RowHist {
     unsigned int cnt[kRowBins];
-    unsigned long long wt[kRowBins];
+    unsigned int wt[3][kRowBins];
 };
 
 struct RowShared {
@@ -154,7 +158,7 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
         RowHist &h = sh.hist[b];
         for (int i = tid; i < kRowBins; i += blockDim.x) {
             h.cnt[i] = 0;
-            if (kMass) h.wt[i] = 0;
+            if (kMass) h.wt[0][i] = h.wt[1][i] = h.wt[2][i] = 0;
         }
         __syncthreads();
         const uint32_t prefix = sh.prefix, pmask = sh.pmask;
@@ -180,15 +184,29 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
             const bool uniform = __all_sync(0xffffffffu, !in || bin == bin0);
             if (uniform) {
                 if (kMass) {
-                    unsigned long long s = wv;
+                    // chunk sums of the warp (each below 2^21), added once
+                    unsigned int c0 = (unsigned)(wv & 0xffffu), c1 = (unsigned)((wv >> 16) & 0xffffu),
+                                 c2 = (unsigned)(wv >> 32);
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                    if (lane == first) atomicAdd(&h.wt[bin0], s);
+                    for (int o = 16; o > 0; o >>= 1) {
+                        c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+                        c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+                        c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+                    }
+                    if (lane == first) {
+                        atomicAdd(&h.wt[0][bin0], c0);
+                        atomicAdd(&h.wt[1][bin0], c1);
+                        atomicAdd(&h.wt[2][bin0], c2);
+                    }
                 }
                 if (lane == first) atomicAdd(&h.cnt[bin0], (unsigned)__popc(active));
             } else if (in) {
                 atomicAdd(&h.cnt[bin], 1u);
-                if (kMass) atomicAdd(&h.wt[bin], wv);
+                if (kMass) {
+                    atomicAdd(&h.wt[0][bin], (unsigned)(wv & 0xffffu));
+                    atomicAdd(&h.wt[1][bin], (unsigned)((wv >> 16) & 0xffffu));
+                    atomicAdd(&h.wt[2][bin], (unsigned)(wv >> 32));
+                }
             }
         }
         rc.cl.sync();
@@ -200,7 +218,9 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
                 if (r < rc.nranks) {
                     const RowHist &rh = rc.cl.map_shared_rank(&sh, r)->hist[b];
                     c += rh.cnt[i];
-                    if (kMass) w += rh.wt[i];
+                    if (kMass)
+                        w += (unsigned long long)rh.wt[0][i] + ((unsigned long long)rh.wt[1][i] << 16) +
+                             ((unsigned long long)rh.wt[2][i] << 32);
                 }
             }
             sh.gcnt[i] = c;

@@ -82,6 +82,7 @@ struct Ctrl {
     uint32_t kvstage[2][8];           // producer: their readable-key masks
     uint32_t vstage[2][kMaxBlocks / 32];  // producer: their visible-block masks
     TileInfo tinfo[2];                // producer: decoded current and next tile
+    float colstage[4][2][kCols];      // producer: staged (lse, q_pos bits) of upcoming column blocks
 };
 
 struct TcArgs {
@@ -340,10 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             int64_t tid;
             int n, page, kp[8];
         };
-        struct ColRaw {
-            float l[4];
-            int p[4];
-        };
         auto issue_tile = [&](int64_t tid, TileRaw &r) {
             r.tid = tid;
             if (tid >= a.total_tiles) return;
@@ -454,14 +451,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return -1;
         };
-        auto issue_cols = [&](const TileInfo &f, int b, ColRaw &cr) {
+        // Column data (lse, q_pos) of a block, copied asynchronously into a staging slot of shared memory
+        // (cp.async: no register waits on the copies); one commit group per call, possibly empty.
+        // Slots in use at any time: the current block's, the next tile's first block's, and the one being
+        // filled for the next block of this tile; a new slot is any other of the four.
+        auto pick_slot = [](uint32_t x, uint32_t y) -> uint32_t {
+            uint32_t s = 0;
+            while (s == x || s == y) ++s;
+            return s;
+        };
+        auto issue_cols = [&](const TileInfo *f, int b, uint32_t slot) -> uint32_t {
+            if (f != nullptr) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int col = u * 32 + lane, jl = col / G, g = col % G;
-                const int j = min(b * nqb + jl, a.q.max_q - 1);
-                cr.l[u] = a.q.lse[((int64_t)(f.seq * c.num_layers + f.layer) * Hq + f.kvh * G + g) * a.q.max_q + j];
-                cr.p[u] = a.q.q_pos[(int64_t)f.seq * a.q.max_q + j];
+                for (int u = 0; u < 4; ++u) {
+                    const int col = u * 32 + lane, jl = col / G, g = col % G;
+                    const int j = min(b * nqb + jl, a.q.max_q - 1);
+                    const float *ls =
+                        a.q.lse + ((int64_t)(f->seq * c.num_layers + f->layer) * Hq + f->kvh * G + g) * a.q.max_q + j;
+                    const int32_t *ps = a.q.q_pos + (int64_t)f->seq * a.q.max_q + j;
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&ctl.colstage[slot][0][col])),
+                                 "l"(ls)
+                                 : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&ctl.colstage[slot][1][col])),
+                                 "l"(ps)
+                                 : "memory");
+                }
             }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            return slot;
         };
         auto fill_tile_part = [&](Item &it, const TileInfo &f, int parity, int flags) {
 #pragma unroll
@@ -476,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 
         TileRaw raw;
-        ColRaw ccur, cnxt;
+        uint32_t cslot = 0, nslot = 0;  // staging slots of the current block and of the next tile's first block
         int par = 0;
         int64_t tid_next = blockIdx.x;
         // find the first tile with keys
@@ -486,10 +503,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tid_next += gridDim.x;
             have = make_info(raw, par);
         }
-        if (have && ctl.tinfo[par].first_vis >= 0) issue_cols(ctl.tinfo[par], ctl.tinfo[par].first_vis, cnxt);
+        nslot = issue_cols(have && ctl.tinfo[par].first_vis >= 0 ? &ctl.tinfo[par] : nullptr, ctl.tinfo[par].first_vis, 0);
         if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
         while (ok && have) {
-            ccur = cnxt;
+            cslot = nslot;
             const int cpar = par;
             const TileInfo &cur = ctl.tinfo[cpar];
             // decode the following tile now (its loads were issued a tile ago) and issue its first columns
@@ -501,7 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
                 have = make_info(r, par);
             }
-            if (have && ctl.tinfo[par].first_vis >= 0) issue_cols(ctl.tinfo[par], ctl.tinfo[par].first_vis, cnxt);
+            nslot = issue_cols(have && ctl.tinfo[par].first_vis >= 0 ? &ctl.tinfo[par] : nullptr,
+                               ctl.tinfo[par].first_vis, pick_slot(cslot, cslot));
 
             if (cur.first_vis < 0) {
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
@@ -534,8 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int b = cur.first_vis; b >= 0;) {
                 const int bn = next_visible(cpar, b);
-                ColRaw cn;
-                if (bn >= 0) issue_cols(cur, bn, cn);
+                const uint32_t bslot = issue_cols(bn >= 0 ? &cur : nullptr, bn, pick_slot(cslot, nslot));
                 // Q block b
                 if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 if (lane == 0) {
@@ -554,20 +571,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int flags = (b == cur.first_vis ? kFirst : 0) | (b == cur.last_vis ? kLast : 0);
                 if (flags & kFirst) fill_tile_part(it, cur, cpar, flags);
                 const int vq = min(nqb, cur.nq - b * nqb);
+                // this block's staged columns have landed: in a tile's first block the next tile's group (issued at
+                // the tile start) and the one just issued may stay in flight, later only the one just issued
+                if (b == cur.first_vis)
+                    asm volatile("cp.async.wait_group 2;" ::: "memory");
+                else
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                __syncwarp();
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int col = u * 32 + lane, jl = col / G;
                     float Lv = INFINITY;
                     int Pv = INT32_MIN;
                     if (jl < vq) {
-                        const float l = ccur.l[u];
+                        const float l = ctl.colstage[cslot][0][col];
                         if (l == -INFINITY) {
                             // a column that saw no key contributes nothing
                         } else if (!is_finite(l)) {
                             report(a.status, KVC_DEV_NONFINITE, cur.row);
                         } else {
                             Lv = l * 1.4426950408889634f;
-                            Pv = ccur.p[u];
+                            Pv = __float_as_int(ctl.colstage[cslot][1][col]);
                         }
                     }
                     it.L[col] = Lv;
@@ -595,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
                 b = bn;
-                ccur = cn;
+                cslot = bslot;
             }
         }
         // end-of-work marker

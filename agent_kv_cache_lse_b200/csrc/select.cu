@@ -27,7 +27,7 @@ struct SelectArgs {
     int slice_cap;
 };
 
-__global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RowShared &sh = *reinterpret_cast<RowShared *>(smem_raw);
     uint32_t *kc = reinterpret_cast<uint32_t *>(smem_raw + sizeof(RowShared));

@@ -142,6 +142,15 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "NVML every 2 ms during the timed steps"}
 
 
+def reduce_over_ranks(total_ms: float, entries: int, device):
+    """Whole-job timing across replicas: the slowest rank's device time and the entries of all ranks."""
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    e = torch.tensor([entries], dtype=torch.int64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(e, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item()), int(e.item())
+
+
 def build_workload(device):
     from agent_kv_cache_lse_b200 import kvc, synth
     spec = synth.llama8b_layer()
@@ -245,10 +254,9 @@ def run_ours(args, rank, world, device):
         score_ms = [evs[k][1].elapsed_time(evs[k][2]) for k in range(args.steps)]
         ratchet_ms = [evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)]
     total_ms = float(sum(step_ms))
+    entries_all = work["entries"] * world
     if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms, entries_all = reduce_over_ranks(total_ms, work["entries"], device)
     assert rnd.device_status()[0] == 0
 
     # end to end through the same public calls with host buffers: H2D inputs, path, D2H results
@@ -260,7 +268,7 @@ def run_ours(args, rank, world, device):
     if rank != 0:
         return None
     ms_step = total_ms / args.steps
-    value = work["entries"] * world / (total_ms / 1e3 / args.steps)
+    value = entries_all / (total_ms / 1e3 / args.steps)
     score_avg = float(np.mean(score_ms))
     achieved = work["flops"] / (score_avg / 1e3) / 1e12
     bytes_step = work["kv_bytes"] + work["meta_bytes"] + work["q_bytes"] + work["logits_bytes"]
