@@ -61,6 +61,13 @@ struct ConfArgs {
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// 2^x by the MUFU unit (ex2.approx, relative error ~2^-22): ample for the log-sum-exp of a step.
+__device__ __forceinline__ float exp2f_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Descending sort of 64 values held two per lane (lane l holds v[0] = x[l], v[1] = x[l + 32]) with a
 // bitonic network over the warp.
 __device__ __forceinline__ void warp_sort64_desc(float &a, float &b) {
@@ -194,7 +201,7 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
     if (cmax != -INFINITY) {
         for (int i = tid; i < cnt; i += kThreads) {
             const float z = zs[i];
-            part += expf(z - cmax);
+            part += exp2f_fast((z - cmax) * 1.4426950408889634f);
             if (z >= tau0) {
                 const int at = atomicAdd(&sh.ncand, 1);
                 if (at < 64) sh.cand[at] = z;

@@ -9,19 +9,26 @@
 //   s[row][i] = sum_{j, g} [q_pos_j >= slot_pos_i] * 2^( (q_{j,g} . k_i) * log2(e)/sqrt(D)
 //                                                      - lse_{j,g} * log2(e) )
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 18 warps):
 //   warp 0     producer: per 256-key tile, 16 TMA page loads (one 16x64 bf16 box per
 //              page and 64-column half of D) gather the K tile from the paged pool into
 //              a 128B-swizzled A operand; per 128-column block of the query set, TMA
-//              loads of the Q block (4-D map: D, head, query, seq*layer) into a stage
-//              ring; per block it also publishes the columns' (lse*log2e, q_pos) and,
-//              once per tile, the keys' positions, through a metadata ring.
+//              loads of the Q block (4-D map: D, query, head, seq*layer, so that a block
+//              lands head-major: column n = g * nqb + query) into a stage ring.  The
+//              block's raw column data (lse, q_pos) is copied a block ahead with
+//              cp.async into a staging slot; per block the producer converts it (four
+//              columns per lane, 16-byte shared-memory reads and writes, no shuffles)
+//              and publishes it through a metadata ring with the block's q_pos range
+//              and, once per tile, the keys' positions.
 //   warp 1     TMEM owner and MMA issuer: for each block, two M=128 x N=128 x K=D
 //              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) into one of two TMEM
 //              accumulator buffers (4 x 128 of the 512 columns).
-//   warps 2-9  epilogue: thread = key (TMEM lane); tcgen05.ld 32 columns at a time,
-//              x = acc * log2e/sqrt(D) - L_col, causal select, ex2, sum in registers.
-//              No cross-thread reduction; one coalesced store per key per tile.
+//   warps 2-17 epilogue: (TMEM lane quadrant, key half, column half); thread = key;
+//              tcgen05.ld 32 columns at a time, x = acc * log2e/sqrt(D) - lse_col * log2e
+//              in packed f32x2 arithmetic, causal select, 2^x (half on the MUFU unit,
+//              half by polynomial on the FMA pipes), sums in registers.  The two column
+//              halves of a key are added through shared memory at the end of the tile;
+//              one coalesced store per key per tile.
 // Blocks whose queries all precede the tile's first key are skipped entirely
 // (no load, no MMA, no epilogue work).  Every barrier wait is bounded (about one
 // second of global time); on expiry the kernel records KVC_DEV_TIMEOUT, drains its
@@ -50,21 +57,27 @@ constexpr int kEpiWarps = 16;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 struct alignas(16) Item {
-    float L[kCols];                     // lse * log2(e) per column (+inf for an absent column)
+    float nL[kCols];                    // -lse * log2(e) per column (-inf for an absent column)
     int32_t qp[kCols];                  // q_pos per column (INT32_MIN for an absent column)
     int32_t kpos[kTileKeys];            // FIRST items: slot_pos of the tile's keys
     uint32_t kvalid[8];                 // FIRST items: keys that are present and readable
-    int32_t cq_min[4], cq_max[4];       // per 32-column chunk: min/max q_pos of its valid columns
     int32_t row, tile, blk, flags;      // blk < 0: tile with no visible block; row < 0: end of work
-    int32_t n_keys, valid_cols, pad0, pad1;
+    int32_t n_keys, chunks, qmin, qmax; // chunks: bit c set when 32-column chunk c has a present column;
+                                        // qmin/qmax: q_pos range of the block's queries
 };
 static_assert(sizeof(Item) % 16 == 0, "items hold float4-read arrays");
 constexpr int kFirst = 1, kLast = 2;
 
 struct TileInfo {
-    int row, t, seq, layer, kvh, n_keys, first_vis, last_vis, kmin, nq;
+    int row, t, seq, layer, kvh, n_keys, first_vis, last_vis, kmin, nq, sbuf;
     unsigned okmask;
     int page[kPagesPerTile];  // physical page of each of the tile's 16 pages (-1: none or invalid)
+};
+
+// Raw column data of one block as copied from global memory: lse in column order, q_pos by query.
+struct alignas(16) ColStage {
+    float lse[kCols];
+    int32_t qpos[kCols];
 };
 
 struct Ctrl {
@@ -76,13 +89,13 @@ struct Ctrl {
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort;
-    int32_t blk_qmin[kMaxBlocks], blk_qmax[kMaxBlocks];
+    int32_t blk_qmin[2][kMaxBlocks], blk_qmax[2][kMaxBlocks];  // q_pos range per block, two sequences
     float part[2][kTileKeys];
     int32_t kstage[2][kTileKeys];     // producer: key positions of the current and the next tile
     uint32_t kvstage[2][8];           // producer: their readable-key masks
     uint32_t vstage[2][kMaxBlocks / 32];  // producer: their visible-block masks
     TileInfo tinfo[2];                // producer: decoded current and next tile
-    float colstage[4][2][kCols];      // producer: staged (lse, q_pos bits) of upcoming column blocks
+    ColStage colstage[4];             // producer: staged raw column data of upcoming blocks
 };
 
 struct TcArgs {
@@ -91,6 +104,7 @@ struct TcArgs {
     float *scores;
     int32_t *status;
     int accumulate;
+    int vec;           // lse / q_pos rows are 16-byte aligned and nqb % 4 == 0: 16-byte column copies
     int nqb;           // queries per column block (floor(128 / G))
     int tiles_per_row;
     int64_t total_tiles;
@@ -206,37 +220,46 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipes: x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez exchange, derived by
-// exp2_poly.py beside this file: max relative error 7.5e-5); 2^n enters through the exponent bits.
-// x is clamped at -126 so the exponent arithmetic stays in range (the result is then ~1e-38).
-__device__ __forceinline__ float exp2_fma(float x) {
+// 2^x on the FMA pipes for a pair of arguments: x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a
+// degree-3 polynomial whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange, derived by exp2_poly.py beside this file: max relative error 7.5e-5); 2^n enters through the
+// exponent bits.  x is clamped at -126 so the exponent arithmetic stays in range (the result is then
+// ~1e-38).  The floating-point steps run as packed f32x2 operations.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
     constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
                     kC3 = 0.0551716685295105f;
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    x = fmaxf(x, -126.0f);
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    float p = fmaf(kC3, f, kC2);
-    p = fmaf(p, f, kC1);
-    p = fmaf(p, f, kC0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+    float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // One 32-column chunk of a key's accumulator row: x = acc * log2(e)/sqrt(D) - lse_col * log2(e), causal
-// select (unless every column of the chunk sees every key of the warp), 2^x, running sums.  Every
-// fourth column's exponential runs on the FMA pipes to relieve the MUFU unit.
-__device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *L, const int32_t *qp, int kpos,
-                                          float sc, bool fast, float &acc0, float &acc1) {
-    const float4 *L4 = reinterpret_cast<const float4 *>(L);
+// select (unless every column of the chunk sees every key of the warp), 2^x, running sums.  Columns go in
+// pairs through packed f32x2 arithmetic; in each group of four, two exponentials run on the MUFU unit and
+// two on the FMA pipes, which keeps both units busy.  An absent column has -lse = -inf: it adds 0 (MUFU)
+// or 2^-126 (polynomial), both far below any tolerance.
+__device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *nL, const int32_t *qp, int kpos,
+                                          float sc, bool fast, float2 &am, float2 &ap) {
+    const float4 *L4 = reinterpret_cast<const float4 *>(nL);
+    const float2 sc2 = make_float2(sc, sc);
     if (fast) {
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
             const float4 l = L4[c4];
-            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x));
-            acc1 += ex2(fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y));
-            acc0 += ex2(fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z));
-            acc1 += exp2_fma(fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w));
+            const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])),
+                                          sc2, make_float2(l.x, l.y));
+            const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])),
+                                          sc2, make_float2(l.z, l.w));
+            am = __fadd2_rn(am, make_float2(ex2(x01.x), ex2(x01.y)));
+            ap = __fadd2_rn(ap, exp2_fma2(x23));
         }
     } else {
         const int4 *P4 = reinterpret_cast<const int4 *>(qp);
@@ -244,14 +267,16 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *
         for (int c4 = 0; c4 < 8; ++c4) {
             const float4 l = L4[c4];
             const int4 p = P4[c4];
-            const float x0 = fmaf(__uint_as_float(r[4 * c4 + 0]), sc, -l.x);
-            const float x1 = fmaf(__uint_as_float(r[4 * c4 + 1]), sc, -l.y);
-            const float x2 = fmaf(__uint_as_float(r[4 * c4 + 2]), sc, -l.z);
-            const float x3 = fmaf(__uint_as_float(r[4 * c4 + 3]), sc, -l.w);
-            acc0 += ex2(p.x >= kpos ? x0 : -INFINITY);
-            acc1 += ex2(p.y >= kpos ? x1 : -INFINITY);
-            acc0 += ex2(p.z >= kpos ? x2 : -INFINITY);
-            acc1 += ex2(p.w >= kpos ? x3 : -INFINITY);
+            float2 x01 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), sc2,
+                                    make_float2(l.x, l.y));
+            float2 x23 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])), sc2,
+                                    make_float2(l.z, l.w));
+            x01.x = p.x >= kpos ? x01.x : -INFINITY;
+            x01.y = p.y >= kpos ? x01.y : -INFINITY;
+            x23.x = p.z >= kpos ? x23.x : -INFINITY;
+            x23.y = p.w >= kpos ? x23.y : -INFINITY;
+            am = __fadd2_rn(am, make_float2(ex2(x01.x), ex2(x01.y)));
+            ap = __fadd2_rn(ap, exp2_fma2(x23));
         }
     }
 }
@@ -268,6 +293,7 @@ struct Plan {
     static constexpr int kOffItems = kOffB + kStages * kBBytes;
     static constexpr int kOffCtrl = kOffItems + kMeta * (int)sizeof(Item);
     static constexpr int kBytes = kOffCtrl + (int)sizeof(Ctrl) + 1024;  // + alignment slack
+    static_assert(kBytes <= 232448, "shared memory plan exceeds 227 KB per CTA");
 };
 
 // ---------------------------------------------------------------- the kernel
@@ -328,7 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
         uint32_t qs = 0, qph = 0, mk = 0, mph = 0;
         uint32_t ta = 0;  // K tiles loaded so far: buffer ta & 1, use (ta >> 1) of that buffer
-        int cur_seq = -1, nblk = 0, nq = 0;
+        // q_pos ranges of a sequence's blocks live in one of two buffers: the tile being produced and the one
+        // decoded ahead of it may belong to different sequences
+        int cur_seq = -1, nblk = 0, nq = 0, sbuf = 1;
         const uint32_t a_tx_page = 16 * 128;                 // one 16-row, 128-byte box
         const uint32_t q_tx = (uint32_t)(G * nqb) * 128u;    // one Q box per 64-column chunk
         bool ok = true;
@@ -371,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n_keys = min(kTileKeys, n - k0);
             if (seq != cur_seq) {
                 cur_seq = seq;
+                sbuf ^= 1;
                 nq = min(a.q.num_q[seq], a.q.max_q);
                 nblk = (nq + nqb - 1) / nqb;
                 for (int b = lane; b < nblk; b += 32) {
@@ -381,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mn = min(mn, p);
                         mx = max(mx, p);
                     }
-                    ctl.blk_qmin[b] = mn;
-                    ctl.blk_qmax[b] = mx;
+                    ctl.blk_qmin[sbuf][b] = mn;
+                    ctl.blk_qmax[sbuf][b] = mx;
                 }
                 __syncwarp();
             }
@@ -408,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int first_vis = -1, last_vis = -1;
             for (int b0 = 0; b0 < kMaxBlocks; b0 += 32) {
                 const int b = b0 + lane;
-                const bool v = b < nblk && ctl.blk_qmax[b] >= kmin;
+                const bool v = b < nblk && ctl.blk_qmax[sbuf][b] >= kmin;
                 const unsigned m = __ballot_sync(0xffffffffu, v);
                 if (lane == 0) ctl.vstage[parity][b0 >> 5] = m;
                 if (m) {
@@ -435,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 f.last_vis = last_vis;
                 f.kmin = kmin;
                 f.nq = nq;
+                f.sbuf = sbuf;
                 f.okmask = okmask;
             }
             __syncwarp();
@@ -462,34 +492,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto issue_cols = [&](const TileInfo *f, int b, uint32_t slot) -> uint32_t {
             if (f != nullptr) {
+                const int mq = a.q.max_q, j0 = b * nqb;
+                const float *lrow = a.q.lse + ((int64_t)(f->seq * c.num_layers + f->layer) * Hq + f->kvh * G) * mq;
+                const int32_t *prow = a.q.q_pos + (int64_t)f->seq * mq;
+                ColStage &cs = ctl.colstage[slot];
+                if (a.vec) {
+                    // 16-byte pieces: lse in column order (head-major), then q_pos; pieces past max_q read nothing
+                    if (lane < G * nqb / 4) {
+                        const int col = lane * 4, g = col / nqb, j = j0 + col % nqb;
+                        const int avail = max(0, min(4, mq - j)) * 4;
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(&cs.lse[col])),
+                                     "l"(lrow + (int64_t)g * mq + (avail ? j : 0)), "r"(avail)
+                                     : "memory");
+                    }
+                    if (lane < nqb / 4) {
+                        const int j = j0 + lane * 4;
+                        const int avail = max(0, min(4, mq - j)) * 4;
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(&cs.qpos[lane * 4])),
+                                     "l"(prow + (avail ? j : 0)), "r"(avail)
+                                     : "memory");
+                    }
+                } else {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int col = u * 32 + lane, jl = col / G, g = col % G;
-                    const int j = min(b * nqb + jl, a.q.max_q - 1);
-                    const float *ls =
-                        a.q.lse + ((int64_t)(f->seq * c.num_layers + f->layer) * Hq + f->kvh * G + g) * a.q.max_q + j;
-                    const int32_t *ps = a.q.q_pos + (int64_t)f->seq * a.q.max_q + j;
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&ctl.colstage[slot][0][col])),
-                                 "l"(ls)
-                                 : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&ctl.colstage[slot][1][col])),
-                                 "l"(ps)
-                                 : "memory");
+                    for (int u = 0; u < 4; ++u) {
+                        const int col = u * 32 + lane;
+                        if (col < G * nqb) {
+                            const int g = col / nqb, j = min(j0 + col % nqb, mq - 1);
+                            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&cs.lse[col])),
+                                         "l"(lrow + (int64_t)g * mq + j)
+                                         : "memory");
+                        }
+                        if (col < nqb) {
+                            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&cs.qpos[col])),
+                                         "l"(prow + min(j0 + col, mq - 1))
+                                         : "memory");
+                        }
+                    }
                 }
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
             return slot;
         };
-        auto fill_tile_part = [&](Item &it, const TileInfo &f, int parity, int flags) {
+        // This lane's four columns of every block: 4*lane .. 4*lane+3, query index within the block (or -1
+        // for a column past the group's G*nqb).  With nqb % 4 == 0 the four share one head.
+        int cjl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int col = 4 * lane + i;
+            cjl[i] = col < G * nqb ? col % nqb : -1;
+        }
+        const bool q4 = (nqb & 3) == 0;
+        auto fill_tile_part = [&](Item &it, int parity) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) it.kpos[i * 32 + lane] = ctl.kstage[parity][i * 32 + lane];
             if (lane < 8) it.kvalid[lane] = ctl.kvstage[parity][lane];
-            if (lane == 0) {
-                it.row = f.row;
-                it.tile = f.t;
-                it.n_keys = f.n_keys;
-                it.flags = flags;
-            }
         };
 
         TileRaw raw;
@@ -524,10 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cur.first_vis < 0) {
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
-                fill_tile_part(it, cur, cpar, kFirst | kLast);
+                fill_tile_part(it, cpar);
                 if (lane == 0) {
-                    it.blk = -1;
-                    it.valid_cols = 0;
+                    *reinterpret_cast<int4 *>(&it.row) = make_int4(cur.row, cur.t, -1, kFirst | kLast);
+                    *reinterpret_cast<int4 *>(&it.n_keys) = make_int4(cur.n_keys, 0, INT32_MAX, INT32_MIN);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
@@ -560,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kc = 0; kc < PL::kChunks; ++kc) {
                         const uint32_t dst = smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128));
-                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, cur.kvh * G, b * nqb,
+                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, b * nqb, cur.kvh * G,
                                     cur.seq * c.num_layers + cur.layer);
                     }
                 }
@@ -569,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
                 const int flags = (b == cur.first_vis ? kFirst : 0) | (b == cur.last_vis ? kLast : 0);
-                if (flags & kFirst) fill_tile_part(it, cur, cpar, flags);
+                if (flags & kFirst) fill_tile_part(it, cpar);
                 const int vq = min(nqb, cur.nq - b * nqb);
                 // this block's staged columns have landed: in a tile's first block the next tile's group (issued at
                 // the tile start) and the one just issued may stay in flight, later only the one just issued
@@ -578,42 +634,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else
                     asm volatile("cp.async.wait_group 1;" ::: "memory");
                 __syncwarp();
+                {
+                    // four columns per lane: one 16-byte read of the raw lse, converted, one 16-byte write
+                    const ColStage &cs = ctl.colstage[cslot];
+                    const float4 lr = *reinterpret_cast<const float4 *>(&cs.lse[4 * lane]);
+                    int4 qv;
+                    if (q4 && cjl[0] >= 0) {
+                        qv = *reinterpret_cast<const int4 *>(&cs.qpos[cjl[0]]);
+                    } else {
+                        qv.x = cjl[0] >= 0 ? cs.qpos[cjl[0]] : 0;
+                        qv.y = cjl[1] >= 0 ? cs.qpos[cjl[1]] : 0;
+                        qv.z = cjl[2] >= 0 ? cs.qpos[cjl[2]] : 0;
+                        qv.w = cjl[3] >= 0 ? cs.qpos[cjl[3]] : 0;
+                    }
+                    const float lv[4] = {lr.x, lr.y, lr.z, lr.w};
+                    const int pv[4] = {qv.x, qv.y, qv.z, qv.w};
+                    float nl[4];
+                    int qq[4];
+                    bool any = false;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int col = u * 32 + lane, jl = col / G;
-                    float Lv = INFINITY;
-                    int Pv = INT32_MIN;
-                    if (jl < vq) {
-                        const float l = ctl.colstage[cslot][0][col];
-                        if (l == -INFINITY) {
-                            // a column that saw no key contributes nothing
-                        } else if (!is_finite(l)) {
-                            report(a.status, KVC_DEV_NONFINITE, cur.row);
-                        } else {
-                            Lv = l * 1.4426950408889634f;
-                            Pv = __float_as_int(ctl.colstage[cslot][1][col]);
+                    for (int i = 0; i < 4; ++i) {
+                        nl[i] = -INFINITY;
+                        qq[i] = INT32_MIN;
+                        if (cjl[i] >= 0 && cjl[i] < vq) {
+                            const float l = lv[i];
+                            if (l == -INFINITY) {
+                                // a column that saw no key contributes nothing
+                            } else if (!is_finite(l)) {
+                                report(a.status, KVC_DEV_NONFINITE, cur.row);
+                            } else {
+                                nl[i] = -l * 1.4426950408889634f;
+                                qq[i] = pv[i];
+                                any = true;
+                            }
                         }
                     }
-                    it.L[col] = Lv;
-                    it.qp[col] = Pv;
-                    int mn = Pv == INT32_MIN ? INT32_MAX : Pv, mx = Pv;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    }
+                    *reinterpret_cast<float4 *>(&it.nL[4 * lane]) = make_float4(nl[0], nl[1], nl[2], nl[3]);
+                    *reinterpret_cast<int4 *>(&it.qp[4 * lane]) = make_int4(qq[0], qq[1], qq[2], qq[3]);
+                    const unsigned bal = __ballot_sync(0xffffffffu, any);
                     if (lane == 0) {
-                        it.cq_min[u] = mn;
-                        it.cq_max[u] = mx;
+                        const int chunks = ((bal & 0xFFu) ? 1 : 0) | ((bal & 0xFF00u) ? 2 : 0) |
+                                           ((bal & 0xFF0000u) ? 4 : 0) | ((bal & 0xFF000000u) ? 8 : 0);
+                        *reinterpret_cast<int4 *>(&it.row) = make_int4(cur.row, cur.t, b, flags);
+                        *reinterpret_cast<int4 *>(&it.n_keys) =
+                            make_int4(cur.n_keys, chunks, ctl.blk_qmin[cur.sbuf][b], ctl.blk_qmax[cur.sbuf][b]);
                     }
-                }
-                if (lane == 0) {
-                    it.row = cur.row;
-                    it.tile = cur.t;
-                    it.blk = b;
-                    it.flags = flags;
-                    it.n_keys = cur.n_keys;
-                    it.valid_cols = vq * G;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
@@ -704,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key = half * 128 + quad * 32 + lane;  // key within the tile = TMEM lane of its half
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         uint32_t mk = 0, mph = 0, ab = 0, abph = 0, tcount = 0;
-        float acc0 = 0.f, acc1 = 0.f;
+        float2 am = make_float2(0.f, 0.f), ap = make_float2(0.f, 0.f);
         int kpos = INT32_MAX, wkmin = INT32_MAX, wkmax = INT32_MIN;
         bool kv = false;
         const float sc = a.scale_log2e;
@@ -715,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (row < 0) break;
             const int flags = it.flags, blk = it.blk;
             if (flags & kFirst) {
-                acc0 = acc1 = 0.f;
+                am = ap = make_float2(0.f, 0.f);
                 kv = (it.kvalid[key >> 5] >> (key & 31)) & 1u;
                 kpos = it.kpos[key];
                 int mn = kv ? kpos : INT32_MAX, mx = kv ? kpos : INT32_MIN;
@@ -731,24 +796,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (blk >= 0) {
                 if (!mbar_wait(&ctl.acc_full[ab], abph, ctl, a.status, row)) break;
                 tc_fence_after();
-                const int vcols = it.valid_cols;
+                const int4 hd = *reinterpret_cast<const int4 *>(&it.n_keys);  // n_keys, chunks, qmin, qmax
                 const uint32_t tbase = tmem + lane_addr + ab * 256 + half * kCols + colh * 64;
                 const int ch0 = colh * 2, ch1 = ch0 + 1;
-                // a chunk is skipped when it holds no column or no key of this warp sees any of its columns
-                const bool do0 = ch0 * 32 < vcols && wkmax != INT32_MIN && it.cq_max[ch0] >= wkmin;
-                const bool do1 = ch1 * 32 < vcols && wkmax != INT32_MIN && it.cq_max[ch1] >= wkmin;
+                // a chunk is skipped when it holds no present column or no key of this warp sees any query of
+                // the block; when every query of the block sees every key of the warp, no causal select
+                const bool sees = wkmax != INT32_MIN && hd.w >= wkmin;
+                const bool fast = hd.z >= wkmax;
                 uint32_t r[32];
-                if (do0) {
+                if (sees && ((hd.y >> ch0) & 1)) {
                     tmem_ld32(tbase, r);
                     tmem_ld_wait();
-                    const bool fast = (ch0 + 1) * 32 <= vcols && it.cq_min[ch0] >= wkmax;
-                    epi_chunk(r, it.L + ch0 * 32, it.qp + ch0 * 32, kpos, sc, fast, acc0, acc1);
+                    epi_chunk(r, it.nL + ch0 * 32, it.qp + ch0 * 32, kpos, sc, fast, am, ap);
                 }
-                if (do1) {
+                if (sees && ((hd.y >> ch1) & 1)) {
                     tmem_ld32(tbase + 32, r);
                     tmem_ld_wait();
-                    const bool fast = (ch1 + 1) * 32 <= vcols && it.cq_min[ch1] >= wkmax;
-                    epi_chunk(r, it.L + ch1 * 32, it.qp + ch1 * 32, kpos, sc, fast, acc0, acc1);
+                    epi_chunk(r, it.nL + ch1 * 32, it.qp + ch1 * 32, kpos, sc, fast, am, ap);
                 }
                 tc_fence_before();
                 if (flags & kLast) {
@@ -756,13 +820,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t p = tcount & 1, ph = (tcount >> 1) & 1;
                     ++tcount;
                     if (colh == 1) {
-                        ctl.part[p][key] = acc0 + acc1;
+                        ctl.part[p][key] = (am.x + am.y) + (ap.x + ap.y);
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&ctl.part_full[p]);
                     } else {
                         if (!mbar_wait(&ctl.part_full[p], ph, ctl, a.status, row)) break;
                         if (kv) {
-                            const float v = (acc0 + acc1) + ctl.part[p][key];
+                            const float v = ((am.x + am.y) + (ap.x + ap.y)) + ctl.part[p][key];
                             *dst = a.accumulate ? *dst + v : v;
                         }
                     }
@@ -831,11 +895,12 @@ cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool
         }
     }
     {
-        cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)q.num_q_heads, (cuuint64_t)q.max_q,
+        // dimensions (D, query, head, seq*layer): a box lands head-major, column n = g * nqb + query
+        cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)q.max_q, (cuuint64_t)q.num_q_heads,
                               (cuuint64_t)c.num_seqs * c.num_layers};
-        cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)q.num_q_heads * D * 2,
+        cuuint64_t strides[3] = {(cuuint64_t)q.num_q_heads * D * 2, (cuuint64_t)D * 2,
                                  (cuuint64_t)q.max_q * q.num_q_heads * D * 2};
-        cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)nqb, 1};
+        cuuint32_t box[4] = {64, (cuuint32_t)nqb, (cuuint32_t)G, 1};
         cuuint32_t es[4] = {1, 1, 1, 1};
         CUresult r = enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q.q), dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -851,6 +916,8 @@ cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool
     args.scores = scores;
     args.status = status;
     args.accumulate = accumulate ? 1 : 0;
+    args.vec = ((reinterpret_cast<uintptr_t>(q.lse) | reinterpret_cast<uintptr_t>(q.q_pos)) & 15) == 0 &&
+               q.max_q % 4 == 0 && nqb % 4 == 0;
     args.nqb = nqb;
     args.tiles_per_row = (int)((c.max_slots + kTileKeys - 1) / kTileKeys);
     args.total_tiles = (int64_t)c.rows * args.tiles_per_row;
