@@ -9,21 +9,24 @@
 //   s[row][i] = sum_{j, g} [q_pos_j >= slot_pos_i] * 2^( (q_{j,g} . k_i) * log2(e)/sqrt(D)
 //                                                      - lse_{j,g} * log2(e) )
 //
-// Design (one persistent CTA per SM, 18 warps):
-//   warp 0     producer: per 256-key tile, 16 TMA page loads (one 16x64 bf16 box per
-//              page and 64-column half of D) gather the K tile from the paged pool into
-//              a 128B-swizzled A operand; per 128-column block of the query set, TMA
-//              loads of the Q block (4-D map: D, query, head, seq*layer, so that a block
-//              lands head-major: column n = g * nqb + query) into a stage ring.  The
-//              block's raw column data (lse, q_pos) is copied a block ahead with
-//              cp.async into a staging slot; per block the producer converts it (four
-//              columns per lane, 16-byte shared-memory reads and writes, no shuffles)
-//              and publishes it through a metadata ring with the block's q_pos range
+// Design (one persistent CTA per SM, 19 warps):
+//   warp 2     decoder: per 256-key tile (one tile ahead), the row length, block-table
+//              entries and slot positions, the keys' position range and with it the
+//              visible column blocks; a tile record goes to the TMA warp through a ring.
+//              Per visible 128-column block (query, head) of the query set, the raw column
+//              data (lse, q_pos) is copied a block ahead with cp.async into a staging slot,
+//              converted (four columns per lane, 16-byte shared-memory accesses, no
+//              shuffles) and published through a metadata ring with the block's q_pos range
 //              and, once per tile, the keys' positions.
+//   warp 0     TMA: per tile record, 16 page loads (one 16x64 bf16 box per page and
+//              64-column half of D) gather the K tile from the paged pool into a
+//              128B-swizzled A operand; per visible block, the Q block (4-D map: D, query,
+//              head, seq*layer, so that a block lands head-major: column n = g * nqb + query)
+//              into a stage ring.
 //   warp 1     TMEM owner and MMA issuer: for each block, two M=128 x N=128 x K=D
 //              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) into one of two TMEM
 //              accumulator buffers (4 x 128 of the 512 columns).
-//   warps 2-17 epilogue: (TMEM lane quadrant, key half, column half); thread = key;
+//   warps 3-18 epilogue: (TMEM lane quadrant, key half, column half); thread = key;
 //              tcgen05.ld 32 columns at a time, x = acc * log2e/sqrt(D) - lse_col * log2e
 //              in packed f32x2 arithmetic, causal select, 2^x (half on the MUFU unit,
 //              half by polynomial on the FMA pipes), sums in registers.  The two column
@@ -52,7 +55,8 @@ constexpr int kPagesPerTile = 16;       // page_size 16
 constexpr int kCols = 128;              // MMA N: query columns per block
 constexpr int kMeta = 8;                // metadata ring depth
 constexpr int kMaxBlocks = 256;         // column blocks per sequence
-constexpr int kThreads = 576;           // 18 warps
+constexpr int kTiles = 4;               // tile ring depth (decoder -> TMA warp)
+constexpr int kThreads = 608;           // 19 warps: TMA, MMA, decoder, 16 epilogue
 constexpr int kEpiWarps = 16;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
@@ -68,10 +72,13 @@ struct alignas(16) Item {
 static_assert(sizeof(Item) % 16 == 0, "items hold float4-read arrays");
 constexpr int kFirst = 1, kLast = 2;
 
-struct TileInfo {
-    int row, t, seq, layer, kvh, n_keys, first_vis, last_vis, kmin, nq, sbuf;
-    unsigned okmask;
-    int page[kPagesPerTile];  // physical page of each of the tile's 16 pages (-1: none or invalid)
+// A tile as the TMA warp needs it: where its pages are and which column blocks it loads Q for.
+struct TileRec {
+    int32_t row, seq, layer, kvh;                 // row < 0: end of work
+    uint32_t okmask;                              // pages that are present and readable
+    int32_t first_vis, pad0, pad1;
+    int32_t page[kPagesPerTile];                  // physical page of each of the tile's 16 pages (-1: none)
+    uint32_t vmask[kMaxBlocks / 32];              // visible column blocks
 };
 
 // Raw column data of one block as copied from global memory: lse in column order, q_pos by query.
@@ -86,6 +93,7 @@ struct Ctrl {
     uint64_t acc_full[2], acc_empty[2];
     uint64_t m_full[kMeta], m_empty[kMeta];
     uint64_t part_full[2];                 // column-half partial sums of a tile, double-buffered
+    uint64_t t_full[kTiles], t_empty[kTiles];
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort;
@@ -94,7 +102,7 @@ struct Ctrl {
     int32_t kstage[2][kTileKeys];     // producer: key positions of the current and the next tile
     uint32_t kvstage[2][8];           // producer: their readable-key masks
     uint32_t vstage[2][kMaxBlocks / 32];  // producer: their visible-block masks
-    TileInfo tinfo[2];                // producer: decoded current and next tile
+    TileRec trec[kTiles];             // tile ring
     ColStage colstage[4];             // producer: staged raw column data of upcoming blocks
 };
 
@@ -281,6 +289,19 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *
     }
 }
 
+// Next visible column block after b in a 256-bit mask (-1: none).
+__device__ __forceinline__ int next_visible(const uint32_t *vmask, int b) {
+    for (int x = b + 1; x < kMaxBlocks; ++x) {
+        const uint32_t w = vmask[x >> 5] >> (x & 31);
+        if (w == 0u) {
+            x |= 31;
+            continue;
+        }
+        return x + __ffs(w) - 1;
+    }
+    return -1;
+}
+
 // ---------------------------------------------------------------- shared memory plan
 template <int D>
 struct Plan {
@@ -330,6 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&ctl.m_full[k], 1);
             mbar_init(&ctl.m_empty[k], 1 + kEpiWarps);
         }
+        for (int k = 0; k < kTiles; ++k) {
+            mbar_init(&ctl.t_full[k], 1);
+            mbar_init(&ctl.t_empty[k], 1);
+        }
         mbar_init(&ctl.drain, 1);
         ctl.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -349,25 +374,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int RPS = c.num_layers * c.num_kv_heads;
 
     if (warp == 0) {
-        // ============================== producer ==============================
+        // ============================== TMA loads ==============================
+        // Follows the tile ring: per tile, the K tile into the free A buffer, then the Q block of every visible
+        // column block into the stage ring, in the order the MMA warp consumes them.
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
-        uint32_t qs = 0, qph = 0, mk = 0, mph = 0;
+        uint32_t qs = 0, qph = 0, tk = 0, tph = 0;
         uint32_t ta = 0;  // K tiles loaded so far: buffer ta & 1, use (ta >> 1) of that buffer
-        // q_pos ranges of a sequence's blocks live in one of two buffers: the tile being produced and the one
-        // decoded ahead of it may belong to different sequences
-        int cur_seq = -1, nblk = 0, nq = 0, sbuf = 1;
         const uint32_t a_tx_page = 16 * 128;                 // one 16-row, 128-byte box
         const uint32_t q_tx = (uint32_t)(G * nqb) * 128u;    // one Q box per 64-column chunk
         bool ok = true;
-        // ---- tile bookkeeping, prefetched one tile ahead.  Raw loads (row length, the tile's block-table
-        // entries and slot positions, and the first visible block's column data) are issued a whole tile
-        // before they are used, and nothing branches on a loaded value until then.
+        for (;;) {
+            if (!mbar_wait(&ctl.t_full[tk], tph, ctl, a.status, -1)) { ok = false; break; }
+            const TileRec &R = ctl.trec[tk];
+            const int row = R.row;
+            if (row < 0) break;
+            const int zq = R.seq * c.num_layers + R.layer, hq0 = R.kvh * G, first_vis = R.first_vis;
+            const unsigned okmask = R.okmask;
+            const int my_page = lane < kPagesPerTile ? R.page[lane] : -1;
+            // K tile into the free buffer: one box per (page, 64-column chunk)
+            const uint32_t abuf = ta & 1;
+            if (!mbar_wait(&ctl.a_empty[abuf], ((ta >> 1) & 1) ^ 1, ctl, a.status, row)) { ok = false; break; }
+            ++ta;
+            if (lane == 0) mbar_expect_tx(&ctl.a_full[abuf], (uint32_t)__popc(okmask) * a_tx_page * PL::kChunks);
+            __syncwarp();
+            if (my_page >= 0) {
+                const int half = lane >> 3, r0 = (lane & 7) * 16;
+#pragma unroll
+                for (int kc = 0; kc < PL::kChunks; ++kc) {
+                    const uint32_t dst =
+                        smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
+                    tma_load_2d(dst, &tmap_k, &ctl.a_full[abuf], kc * 64, my_page * 16);
+                }
+            }
+            // Q blocks of the visible column blocks
+            for (int b = first_vis; b >= 0; b = next_visible(R.vmask, b)) {
+                if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, row)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_expect_tx(&ctl.q_full[qs], q_tx * PL::kChunks);
+#pragma unroll
+                    for (int kc = 0; kc < PL::kChunks; ++kc) {
+                        const uint32_t dst = smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128));
+                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, b * nqb, hq0, zq);
+                    }
+                }
+                __syncwarp();
+                if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
+            }
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(&ctl.t_empty[tk]);
+            if (++tk == kTiles) { tk = 0; tph ^= 1; }
+        }
+        if (!ok || ctl.abort) {
+            // drain our own copies before the CTA can exit: every issued TMA phase completes
+            for (int s = 0; s < PL::kStages; ++s) {
+                const uint64_t t0 = now_ns();
+                while (!mbar_test(&ctl.q_full[s], (qph ^ (s < (int)qs ? 0u : 1u)) & 1u) && now_ns() - t0 < kTimeoutNs) {}
+            }
+            for (uint32_t b = 0; b < 2; ++b) {
+                const uint32_t fills = (ta + 1 - b) / 2;  // loads that went to buffer b
+                if (fills == 0) continue;
+                const uint64_t t0 = now_ns();
+                while (!mbar_test(&ctl.a_full[b], (fills - 1) & 1) && now_ns() - t0 < kTimeoutNs) {}
+            }
+        }
+    } else if (warp == 2) {
+        // ============================== tiles and column data ==============================
+        // Decodes each tile one tile ahead (row length, block-table entries, slot positions, visible column
+        // blocks) and hands it to the TMA warp through the tile ring; copies every visible block's raw column
+        // data a block ahead with cp.async; converts it and publishes one metadata item per block.
+        uint32_t mk = 0, mph = 0, tk = 0, tph = 0;
+        // q_pos ranges of a sequence's blocks live in one of two buffers: the tile being produced and the one
+        // decoded ahead of it may belong to different sequences
+        int cur_seq = -1, nblk = 0, nq = 0, sbuf = 1;
+        bool ok = true;
         const int mp = c.max_pages_per_row;
         const int64_t ms = c.max_slots;
+        // Raw loads of a tile (row length, its block-table entries and slot positions), issued a whole tile
+        // before they are used; nothing branches on a loaded value until then.
         struct TileRaw {
             int64_t tid;
             int n, page, kp[8];
+        };
+        // A decoded tile, held in registers.
+        struct Tile {
+            int row, t, n_keys, first_vis, last_vis, nq, sbuf;
+            const float *lrow;    // lse of the group's first head (sequence, layer, KV head)
+            const int32_t *prow;  // q_pos of the sequence
         };
         auto issue_tile = [&](int64_t tid, TileRaw &r) {
             r.tid = tid;
@@ -381,9 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i)
                 r.kp[i] = c.slot_pos[row * ms + min((int64_t)t * kTileKeys + i * 32 + lane, ms - 1)];
         };
-        // Decode a tile (waits for its raw loads).  Returns false for a tile with no keys.
-        auto make_info = [&](const TileRaw &r, int parity) -> bool {
-            TileInfo &f = ctl.tinfo[parity];
+        // Decode a tile (waits for its raw loads) into T and key staging buffer `parity`; a tile with a visible
+        // block also goes to the TMA warp.  Returns false for a tile with no keys (or on abort, with ok cleared).
+        auto make_tile = [&](const TileRaw &r, int parity, Tile &T) -> bool {
             if (r.tid >= a.total_tiles) return false;
             const int64_t rr = r.tid % RPS, rest = r.tid / RPS;
             const int t = (int)(rest % a.tiles_per_row);
@@ -420,7 +513,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 page_ok = r.page >= 0 && r.page < c.num_pages;
                 if (!page_ok) report(a.status, KVC_DEV_BAD_PAGE, row);
             }
-            if (lane < kPagesPerTile) f.page[lane] = page_ok ? r.page : -1;
             const unsigned okmask = __ballot_sync(0xffffffffu, page_ok);
             int kmin = INT32_MAX;
 #pragma unroll
@@ -435,14 +527,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
             // visible blocks: some query at or after the tile's first key position
             int first_vis = -1, last_vis = -1;
-            for (int b0 = 0; b0 < kMaxBlocks; b0 += 32) {
-                const int b = b0 + lane;
+#pragma unroll
+            for (int w = 0; w < kMaxBlocks / 32; ++w) {
+                const int b = w * 32 + lane;
                 const bool v = b < nblk && ctl.blk_qmax[sbuf][b] >= kmin;
                 const unsigned m = __ballot_sync(0xffffffffu, v);
-                if (lane == 0) ctl.vstage[parity][b0 >> 5] = m;
+                if (lane == 0) ctl.vstage[parity][w] = m;
                 if (m) {
-                    if (first_vis < 0) first_vis = b0 + __ffs(m) - 1;
-                    last_vis = b0 + 31 - __clz(m);
+                    if (first_vis < 0) first_vis = w * 32 + __ffs(m) - 1;
+                    last_vis = w * 32 + 31 - __clz(m);
                 }
             }
             if (lane < 8) {
@@ -453,33 +546,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ctl.kvstage[parity][lane] = w;
             }
-            if (lane == 0) {
-                f.row = row;
-                f.t = t;
-                f.seq = seq;
-                f.layer = (int)(rr / c.num_kv_heads);
-                f.kvh = (int)(rr % c.num_kv_heads);
-                f.n_keys = n_keys;
-                f.first_vis = first_vis;
-                f.last_vis = last_vis;
-                f.kmin = kmin;
-                f.nq = nq;
-                f.sbuf = sbuf;
-                f.okmask = okmask;
-            }
+            const int layer = (int)(rr / c.num_kv_heads), kvh = (int)(rr % c.num_kv_heads);
+            T.row = row;
+            T.t = t;
+            T.n_keys = n_keys;
+            T.first_vis = first_vis;
+            T.last_vis = last_vis;
+            T.nq = nq;
+            T.sbuf = sbuf;
+            T.lrow = a.q.lse + ((int64_t)(seq * c.num_layers + layer) * Hq + kvh * G) * a.q.max_q;
+            T.prow = a.q.q_pos + (int64_t)seq * a.q.max_q;
             __syncwarp();
-            return true;
-        };
-        auto next_visible = [&](int parity, int b) -> int {
-            for (int x = b + 1; x < kMaxBlocks; ++x) {
-                const uint32_t w = ctl.vstage[parity][x >> 5] >> (x & 31);
-                if (w == 0u) {
-                    x = (x | 31);
-                    continue;
+            if (first_vis >= 0) {
+                if (!mbar_wait(&ctl.t_empty[tk], tph ^ 1, ctl, a.status, row)) {
+                    ok = false;
+                    return false;
                 }
-                return x + __ffs(w) - 1;
+                TileRec &R = ctl.trec[tk];
+                if (lane < kPagesPerTile) R.page[lane] = page_ok ? r.page : -1;
+                if (lane < kMaxBlocks / 32) R.vmask[lane] = ctl.vstage[parity][lane];
+                if (lane == 0) {
+                    R.row = row;
+                    R.seq = seq;
+                    R.layer = layer;
+                    R.kvh = kvh;
+                    R.okmask = okmask;
+                    R.first_vis = first_vis;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.t_full[tk]);
+                if (++tk == kTiles) { tk = 0; tph ^= 1; }
             }
-            return -1;
+            return true;
         };
         // Column data (lse, q_pos) of a block, copied asynchronously into a staging slot of shared memory
         // (cp.async: no register waits on the copies); one commit group per call, possibly empty.
@@ -490,11 +588,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (s == x || s == y) ++s;
             return s;
         };
-        auto issue_cols = [&](const TileInfo *f, int b, uint32_t slot) -> uint32_t {
-            if (f != nullptr) {
+        auto issue_cols = [&](const Tile &f, bool valid, int b, uint32_t slot) -> uint32_t {
+            if (valid) {
                 const int mq = a.q.max_q, j0 = b * nqb;
-                const float *lrow = a.q.lse + ((int64_t)(f->seq * c.num_layers + f->layer) * Hq + f->kvh * G) * mq;
-                const int32_t *prow = a.q.q_pos + (int64_t)f->seq * mq;
                 ColStage &cs = ctl.colstage[slot];
                 if (a.vec) {
                     // 16-byte pieces: lse in column order (head-major), then q_pos; pieces past max_q read nothing
@@ -502,14 +598,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int col = lane * 4, g = col / nqb, j = j0 + col % nqb;
                         const int avail = max(0, min(4, mq - j)) * 4;
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(&cs.lse[col])),
-                                     "l"(lrow + (int64_t)g * mq + (avail ? j : 0)), "r"(avail)
+                                     "l"(f.lrow + (int64_t)g * mq + (avail ? j : 0)), "r"(avail)
                                      : "memory");
                     }
                     if (lane < nqb / 4) {
                         const int j = j0 + lane * 4;
                         const int avail = max(0, min(4, mq - j)) * 4;
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(&cs.qpos[lane * 4])),
-                                     "l"(prow + (avail ? j : 0)), "r"(avail)
+                                     "l"(f.prow + (avail ? j : 0)), "r"(avail)
                                      : "memory");
                     }
                 } else {
@@ -519,12 +615,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (col < G * nqb) {
                             const int g = col / nqb, j = min(j0 + col % nqb, mq - 1);
                             asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&cs.lse[col])),
-                                         "l"(lrow + (int64_t)g * mq + j)
+                                         "l"(f.lrow + (int64_t)g * mq + j)
                                          : "memory");
                         }
                         if (col < nqb) {
                             asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&cs.qpos[col])),
-                                         "l"(prow + min(j0 + col, mq - 1))
+                                         "l"(f.prow + min(j0 + col, mq - 1))
                                          : "memory");
                         }
                     }
@@ -549,33 +645,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 
         TileRaw raw;
+        Tile cur{}, nxt{};
         uint32_t cslot = 0, nslot = 0;  // staging slots of the current block and of the next tile's first block
         int par = 0;
         int64_t tid_next = blockIdx.x;
         // find the first tile with keys
         bool have = false;
-        while (!have && tid_next < a.total_tiles) {
+        while (ok && !have && tid_next < a.total_tiles) {
             issue_tile(tid_next, raw);
             tid_next += gridDim.x;
-            have = make_info(raw, par);
+            have = make_tile(raw, par, nxt);
         }
-        nslot = issue_cols(have && ctl.tinfo[par].first_vis >= 0 ? &ctl.tinfo[par] : nullptr, ctl.tinfo[par].first_vis, 0);
+        nslot = issue_cols(nxt, ok && have && nxt.first_vis >= 0, nxt.first_vis, 0);
         if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
         while (ok && have) {
+            cur = nxt;
             cslot = nslot;
             const int cpar = par;
-            const TileInfo &cur = ctl.tinfo[cpar];
             // decode the following tile now (its loads were issued a tile ago) and issue its first columns
             par ^= 1;
             have = false;
-            while (!have && tid_next < a.total_tiles) {
+            while (ok && !have && tid_next < a.total_tiles) {
                 const TileRaw r = raw;
                 tid_next += gridDim.x;
                 if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
-                have = make_info(r, par);
+                have = make_tile(r, par, nxt);
             }
-            nslot = issue_cols(have && ctl.tinfo[par].first_vis >= 0 ? &ctl.tinfo[par] : nullptr,
-                               ctl.tinfo[par].first_vis, pick_slot(cslot, cslot));
+            if (!ok) break;
+            nslot = issue_cols(nxt, have && nxt.first_vis >= 0, nxt.first_vis, pick_slot(cslot, cslot));
 
             if (cur.first_vis < 0) {
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
@@ -590,38 +687,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
                 continue;
             }
-            // K tile into the free buffer: one box per (page, 64-column chunk)
-            const uint32_t abuf = ta & 1;
-            if (!mbar_wait(&ctl.a_empty[abuf], ((ta >> 1) & 1) ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
-            ++ta;
-            if (lane == 0) mbar_expect_tx(&ctl.a_full[abuf], (uint32_t)__popc(cur.okmask) * a_tx_page * PL::kChunks);
-            __syncwarp();
-            const int my_page = lane < kPagesPerTile ? cur.page[lane] : -1;
-            if (my_page >= 0) {
-                const int half = lane >> 3, r0 = (lane & 7) * 16;
-#pragma unroll
-                for (int kc = 0; kc < PL::kChunks; ++kc) {
-                    const uint32_t dst =
-                        smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + half * (128 * 128) + r0 * 128);
-                    tma_load_2d(dst, &tmap_k, &ctl.a_full[abuf], kc * 64, my_page * 16);
-                }
-            }
             for (int b = cur.first_vis; b >= 0;) {
-                const int bn = next_visible(cpar, b);
-                const uint32_t bslot = issue_cols(bn >= 0 ? &cur : nullptr, bn, pick_slot(cslot, nslot));
-                // Q block b
-                if (!mbar_wait(&ctl.q_empty[qs], qph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_expect_tx(&ctl.q_full[qs], q_tx * PL::kChunks);
-#pragma unroll
-                    for (int kc = 0; kc < PL::kChunks; ++kc) {
-                        const uint32_t dst = smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128));
-                        tma_load_4d(dst, &tmap_q, &ctl.q_full[qs], kc * 64, b * nqb, cur.kvh * G,
-                                    cur.seq * c.num_layers + cur.layer);
-                    }
-                }
-                if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
-                // metadata item (the column data was loaded a block earlier)
+                const int bn = next_visible(ctl.vstage[cpar], b);
+                const uint32_t bslot = issue_cols(cur, bn >= 0, bn, pick_slot(cslot, nslot));
+                // metadata item (the column data was copied a block earlier)
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
                 const int flags = (b == cur.first_vis ? kFirst : 0) | (b == cur.last_vis ? kLast : 0);
@@ -687,26 +756,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cslot = bslot;
             }
         }
-        // end-of-work marker
+        // end-of-work markers: for the MMA and epilogue warps, and for the TMA warp
         if (ok && mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, -1)) {
             if (lane == 0) {
                 items[mk].row = -1;
                 mbar_arrive(&ctl.m_full[mk]);
             }
         }
-        if (!ok || ctl.abort) {
-            // drain our own copies before the CTA can exit: every issued TMA phase completes
-            for (int s = 0; s < PL::kStages; ++s) {
-                const uint64_t t0 = now_ns();
-                while (!mbar_test(&ctl.q_full[s], (qph ^ (s < (int)qs ? 0u : 1u)) & 1u) && now_ns() - t0 < kTimeoutNs) {}
-            }
-            for (uint32_t b = 0; b < 2; ++b) {
-                const uint32_t fills = (ta + 1 - b) / 2;  // loads that went to buffer b
-                if (fills == 0) continue;
-                const uint64_t t0 = now_ns();
-                while (!mbar_test(&ctl.a_full[b], (fills - 1) & 1) && now_ns() - t0 < kTimeoutNs) {}
+        if (ok && mbar_wait(&ctl.t_empty[tk], tph ^ 1, ctl, a.status, -1)) {
+            if (lane == 0) {
+                ctl.trec[tk].row = -1;
+                mbar_arrive(&ctl.t_full[tk]);
             }
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // no copy into shared memory outlives the CTA
     } else if (warp == 1) {
         // ============================== MMA issuer ==============================
         uint32_t qs = 0, qph = 0, mk = 0, mph = 0, ab = 0, abph = 0;
@@ -760,11 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t t0 = now_ns();
             while (!mbar_test(&ctl.drain, 0) && now_ns() - t0 < kTimeoutNs) {}
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 3) {
         // ============================== epilogue ==============================
         // 16 warps: (TMEM lane quadrant = warp % 4, key half, column half); the two column halves of a key
         // are added through shared memory at the end of each tile.
-        const int e = warp - 2;
+        const int e = warp - 3;
         const int quad = warp & 3, half = (e >> 2) & 1, colh = e >> 3;
         const int key = half * 128 + quad * 32 + lane;  // key within the tile = TMEM lane of its half
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
