@@ -27,7 +27,7 @@
 //              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) into one of two TMEM
 //              accumulator buffers (4 x 128 of the 512 columns).
 //   warps 3-18 epilogue: (TMEM lane quadrant, key half, column half); thread = key;
-//              tcgen05.ld 32 columns at a time, x = acc * log2e/sqrt(D) - lse_col * log2e
+//              tcgen05.ld 16 columns at a time (double-buffered), x = acc * log2e/sqrt(D) - lse_col * log2e
 //              in packed f32x2 arithmetic, causal select, 2^x (half on the MUFU unit,
 //              half by polynomial on the FMA pipes), sums in registers.  The two column
 //              halves of a key are added through shared memory at the end of the tile;
@@ -81,6 +81,13 @@ struct TileRec {
     uint32_t vmask[kMaxBlocks / 32];              // visible column blocks
 };
 
+// A tile as the decoder works through it (the current one in registers, the next one in shared memory).
+struct Tile {
+    int row, t, n_keys, first_vis, last_vis, nq, sbuf, pad;
+    const float *lrow;    // lse of the group's first head (sequence, layer, KV head)
+    const int32_t *prow;  // q_pos of the sequence
+};
+
 // Raw column data of one block as copied from global memory: lse in column order, q_pos by query.
 struct alignas(16) ColStage {
     float lse[kCols];
@@ -103,6 +110,7 @@ struct Ctrl {
     uint32_t kvstage[2][8];           // producer: their readable-key masks
     uint32_t vstage[2][kMaxBlocks / 32];  // producer: their visible-block masks
     TileRec trec[kTiles];             // tile ring
+    Tile tnext;                       // decoder: the tile decoded ahead
     ColStage colstage[4];             // producer: staged raw column data of upcoming blocks
 };
 
@@ -209,18 +217,24 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+        "[%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's TMEM loads; naming the registers of the load being waited for keeps the compiler from
+// reading them before the wait.
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -249,18 +263,18 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-// One 32-column chunk of a key's accumulator row: x = acc * log2(e)/sqrt(D) - lse_col * log2(e), causal
-// select (unless every column of the chunk sees every key of the warp), 2^x, running sums.  Columns go in
-// pairs through packed f32x2 arithmetic; in each group of four, two exponentials run on the MUFU unit and
-// two on the FMA pipes, which keeps both units busy.  An absent column has -lse = -inf: it adds 0 (MUFU)
-// or 2^-126 (polynomial), both far below any tolerance.
-__device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *nL, const int32_t *qp, int kpos,
-                                          float sc, bool fast, float2 &am, float2 &ap) {
+// Sixteen columns of a key's accumulator row: x = acc * log2(e)/sqrt(D) - lse_col * log2(e), causal select
+// (unless every column of the block sees every key of the warp), 2^x, running sums.  Columns go in pairs
+// through packed f32x2 arithmetic; in each group of four, two exponentials run on the MUFU unit and two on
+// the FMA pipes.  An absent column has -lse = -inf: it adds 0 (MUFU) or 2^-126 (polynomial), both far below
+// any tolerance.
+__device__ __forceinline__ void epi16(const uint32_t (&r)[16], const float *nL, const int32_t *qp, int kpos, float sc,
+                                      bool fast, float2 &am, float2 &ap) {
     const float4 *L4 = reinterpret_cast<const float4 *>(nL);
     const float2 sc2 = make_float2(sc, sc);
     if (fast) {
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
+        for (int c4 = 0; c4 < 4; ++c4) {
             const float4 l = L4[c4];
             const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])),
                                           sc2, make_float2(l.x, l.y));
@@ -272,7 +286,7 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float *
     } else {
         const int4 *P4 = reinterpret_cast<const int4 *>(qp);
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
+        for (int c4 = 0; c4 < 4; ++c4) {
             const float4 l = L4[c4];
             const int4 p = P4[c4];
             float2 x01 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), sc2,
@@ -456,12 +470,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             int64_t tid;
             int n, page, kp[8];
         };
-        // A decoded tile, held in registers.
-        struct Tile {
-            int row, t, n_keys, first_vis, last_vis, nq, sbuf;
-            const float *lrow;    // lse of the group's first head (sequence, layer, KV head)
-            const int32_t *prow;  // q_pos of the sequence
-        };
         auto issue_tile = [&](int64_t tid, TileRaw &r) {
             r.tid = tid;
             if (tid >= a.total_tiles) return;
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i)
                 r.kp[i] = c.slot_pos[row * ms + min((int64_t)t * kTileKeys + i * 32 + lane, ms - 1)];
         };
-        // Decode a tile (waits for its raw loads) into T and key staging buffer `parity`; a tile with a visible
+        // Decode a tile (waits for its raw loads) into T (shared) and key staging buffer `parity`; a tile with a visible
         // block also goes to the TMA warp.  Returns false for a tile with no keys (or on abort, with ok cleared).
         auto make_tile = [&](const TileRaw &r, int parity, Tile &T) -> bool {
             if (r.tid >= a.total_tiles) return false;
@@ -496,15 +504,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 nq = min(a.q.num_q[seq], a.q.max_q);
                 nblk = (nq + nqb - 1) / nqb;
                 for (int b = lane; b < nblk; b += 32) {
-                    int mn = INT32_MAX, mx = INT32_MIN;
-                    const int j1 = min(nq, (b + 1) * nqb);
-                    for (int j = b * nqb; j < j1; ++j) {
-                        const int p = a.q.q_pos[(int64_t)seq * a.q.max_q + j];
-                        mn = min(mn, p);
-                        mx = max(mx, p);
+                    ctl.blk_qmin[sbuf][b] = INT32_MAX;
+                    ctl.blk_qmax[sbuf][b] = INT32_MIN;
+                }
+                __syncwarp();
+                // q_pos range of every block: coalesced loads, four in flight per lane, shared-memory atomics
+                const int32_t *qrow = a.q.q_pos + (int64_t)seq * a.q.max_q;
+                for (int j0 = 0; j0 < nq; j0 += 128) {
+                    int pv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = j0 + u * 32 + lane;
+                        pv[u] = j < nq ? qrow[j] : 0;
                     }
-                    ctl.blk_qmin[sbuf][b] = mn;
-                    ctl.blk_qmax[sbuf][b] = mx;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = j0 + u * 32 + lane;
+                        if (j < nq) {
+                            atomicMin(&ctl.blk_qmin[sbuf][j / nqb], pv[u]);
+                            atomicMax(&ctl.blk_qmax[sbuf][j / nqb], pv[u]);
+                        }
+                    }
                 }
                 __syncwarp();
             }
@@ -547,15 +567,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ctl.kvstage[parity][lane] = w;
             }
             const int layer = (int)(rr / c.num_kv_heads), kvh = (int)(rr % c.num_kv_heads);
-            T.row = row;
-            T.t = t;
-            T.n_keys = n_keys;
-            T.first_vis = first_vis;
-            T.last_vis = last_vis;
-            T.nq = nq;
-            T.sbuf = sbuf;
-            T.lrow = a.q.lse + ((int64_t)(seq * c.num_layers + layer) * Hq + kvh * G) * a.q.max_q;
-            T.prow = a.q.q_pos + (int64_t)seq * a.q.max_q;
+            if (lane == 0) {
+                T.row = row;
+                T.t = t;
+                T.n_keys = n_keys;
+                T.first_vis = first_vis;
+                T.last_vis = last_vis;
+                T.nq = nq;
+                T.sbuf = sbuf;
+                T.lrow = a.q.lse + ((int64_t)(seq * c.num_layers + layer) * Hq + kvh * G) * a.q.max_q;
+                T.prow = a.q.q_pos + (int64_t)seq * a.q.max_q;
+            }
             __syncwarp();
             if (first_vis >= 0) {
                 if (!mbar_wait(&ctl.t_empty[tk], tph ^ 1, ctl, a.status, row)) {
@@ -644,36 +666,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane < 8) it.kvalid[lane] = ctl.kvstage[parity][lane];
         };
 
+        // Tile order: round k takes tiles k * grid .. k * grid + grid - 1, CTA b the b-th of them in even rounds
+        // and the (grid - 1 - b)-th in odd rounds, so that the costly and the cheap ends of the order (under a
+        // causal mask, early positions see more query blocks) share out across CTAs.
+        int64_t round_next = 0;
+        auto next_tid = [&]() -> int64_t {
+            const int64_t k = round_next++;
+            return k * gridDim.x + ((k & 1) ? (int64_t)(gridDim.x - 1 - blockIdx.x) : (int64_t)blockIdx.x);
+        };
         TileRaw raw;
-        Tile cur{}, nxt{};
+        Tile cur{};
+        Tile &nxt = ctl.tnext;
         uint32_t cslot = 0, nslot = 0;  // staging slots of the current block and of the next tile's first block
         int par = 0;
-        int64_t tid_next = blockIdx.x;
+        int64_t tid_next = next_tid();
         // find the first tile with keys
         bool have = false;
         while (ok && !have && tid_next < a.total_tiles) {
             issue_tile(tid_next, raw);
-            tid_next += gridDim.x;
+            tid_next = next_tid();
             have = make_tile(raw, par, nxt);
         }
         nslot = issue_cols(nxt, ok && have && nxt.first_vis >= 0, nxt.first_vis, 0);
         if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
-        while (ok && have) {
-            cur = nxt;
-            cslot = nslot;
-            const int cpar = par;
-            // decode the following tile now (its loads were issued a tile ago) and issue its first columns
+        // Decode the following tile (its loads were issued a tile ago) and copy its first block's columns; done
+        // once the current tile's first item is out, so that the first item does not wait for it.
+        auto decode_next = [&](uint32_t busy) {
             par ^= 1;
             have = false;
             while (ok && !have && tid_next < a.total_tiles) {
                 const TileRaw r = raw;
-                tid_next += gridDim.x;
+                tid_next = next_tid();
                 if (tid_next < a.total_tiles) issue_tile(tid_next, raw);
                 have = make_tile(r, par, nxt);
             }
-            if (!ok) break;
-            nslot = issue_cols(nxt, have && nxt.first_vis >= 0, nxt.first_vis, pick_slot(cslot, cslot));
-
+            nslot = issue_cols(nxt, ok && have && nxt.first_vis >= 0, nxt.first_vis, pick_slot(busy, busy));
+        };
+        while (ok && have) {
+            cur = nxt;
+            cslot = nslot;
+            const int cpar = par;
             if (cur.first_vis < 0) {
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
@@ -685,23 +717,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
+                decode_next(cslot);
                 continue;
             }
+            bool decoded = false, after_decode = false;
             for (int b = cur.first_vis; b >= 0;) {
                 const int bn = next_visible(ctl.vstage[cpar], b);
-                const uint32_t bslot = issue_cols(cur, bn >= 0, bn, pick_slot(cslot, nslot));
+                const uint32_t bslot = issue_cols(cur, bn >= 0, bn, pick_slot(cslot, decoded ? nslot : cslot));
                 // metadata item (the column data was copied a block earlier)
                 if (!mbar_wait(&ctl.m_empty[mk], mph ^ 1, ctl, a.status, cur.row)) { ok = false; break; }
                 Item &it = items[mk];
                 const int flags = (b == cur.first_vis ? kFirst : 0) | (b == cur.last_vis ? kLast : 0);
                 if (flags & kFirst) fill_tile_part(it, cpar);
                 const int vq = min(nqb, cur.nq - b * nqb);
-                // this block's staged columns have landed: in a tile's first block the next tile's group (issued at
-                // the tile start) and the one just issued may stay in flight, later only the one just issued
-                if (b == cur.first_vis)
+                // this block's staged columns have landed; the group just issued may stay in flight, and right after
+                // the next tile's decode so may the next tile's first block (committed between the two)
+                if (after_decode)
                     asm volatile("cp.async.wait_group 2;" ::: "memory");
                 else
                     asm volatile("cp.async.wait_group 1;" ::: "memory");
+                after_decode = false;
                 __syncwarp();
                 {
                     // four columns per lane: one 16-byte read of the raw lse, converted, one 16-byte write
@@ -752,6 +787,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.m_full[mk]);
                 if (++mk == kMeta) { mk = 0; mph ^= 1; }
+                if (!decoded) {
+                    decode_next(bslot);
+                    if (!ok) break;
+                    decoded = after_decode = true;
+                }
                 b = bn;
                 cslot = bslot;
             }
@@ -866,16 +906,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the block; when every query of the block sees every key of the warp, no causal select
                 const bool sees = wkmax != INT32_MIN && hd.w >= wkmin;
                 const bool fast = hd.z >= wkmax;
-                uint32_t r[32];
-                if (sees && ((hd.y >> ch0) & 1)) {
-                    tmem_ld32(tbase, r);
-                    tmem_ld_wait();
-                    epi_chunk(r, it.nL + ch0 * 32, it.qp + ch0 * 32, kpos, sc, fast, am, ap);
-                }
-                if (sees && ((hd.y >> ch1) & 1)) {
-                    tmem_ld32(tbase + 32, r);
-                    tmem_ld_wait();
-                    epi_chunk(r, it.nL + ch1 * 32, it.qp + ch1 * 32, kpos, sc, fast, am, ap);
+                // 16-column TMEM loads, double-buffered: the next one is in flight while the current is summed
+                const bool do0 = sees && ((hd.y >> ch0) & 1), do1 = sees && ((hd.y >> ch1) & 1);
+                const float *nL = it.nL + colh * 64;
+                const int32_t *qp = it.qp + colh * 64;
+                uint32_t ra[16], rb[16];
+                if (do0 && do1) {
+                    tmem_ld16(tbase, ra);
+                    tmem_wait16(ra);
+                    tmem_ld16(tbase + 16, rb);
+                    epi16(ra, nL, qp, kpos, sc, fast, am, ap);
+                    tmem_wait16(rb);
+                    tmem_ld16(tbase + 32, ra);
+                    epi16(rb, nL + 16, qp + 16, kpos, sc, fast, am, ap);
+                    tmem_wait16(ra);
+                    tmem_ld16(tbase + 48, rb);
+                    epi16(ra, nL + 32, qp + 32, kpos, sc, fast, am, ap);
+                    tmem_wait16(rb);
+                    epi16(rb, nL + 48, qp + 48, kpos, sc, fast, am, ap);
+                } else if (do0 || do1) {
+                    const int o = do0 ? 0 : 32;
+                    tmem_ld16(tbase + o, ra);
+                    tmem_wait16(ra);
+                    tmem_ld16(tbase + o + 16, rb);
+                    epi16(ra, nL + o, qp + o, kpos, sc, fast, am, ap);
+                    tmem_wait16(rb);
+                    epi16(rb, nL + o + 16, qp + o + 16, kpos, sc, fast, am, ap);
                 }
                 tc_fence_before();
                 if (flags & kLast) {
