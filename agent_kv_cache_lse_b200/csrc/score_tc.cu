@@ -192,21 +192,24 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// 128B-swizzled K-major operand: 8-row groups 1024 bytes apart, version 1, layout SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
-           ((uint64_t)2 << 61);
-}
+// Shared-memory matrix descriptor of a 128B-swizzled K-major operand (8-row groups 1024 bytes apart, version 1,
+// layout SWIZZLE_128B), split in two words: the high word is the same for every operand here, the low word
+// holds the start address (in 16-byte units, 14 bits) and the leading byte offset (1).  Offsets within one
+// operand buffer are added to the low word directly: addresses stay below 2^18, so the field never carries.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t addr) { return ((addr >> 4) & 0x3FFF) | (1u << 16); }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M = 128, N = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kCols >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+template <bool kAccumulate>
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo) {
+    const uint64_t ad = ((uint64_t)kDescHi << 32) | a_lo, bd = ((uint64_t)kDescHi << 32) | b_lo;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(ad), "l"(bd), "r"(kIdesc), "n"(kAccumulate ? 1 : 0));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -346,6 +349,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const CacheView &c = a.c;
 
+    if (warp == 2 && (int64_t)blockIdx.x < a.total_tiles) {
+        // warm L2 with what the first tile's decode reads (the CTA's first tile has index blockIdx.x): its row
+        // length, block-table entries and slot positions, and the sequence's query count and positions
+        const int RPS0 = c.num_layers * c.num_kv_heads;
+        const int64_t tid = blockIdx.x, rr = tid % RPS0, rest = tid / RPS0;
+        const int t = (int)(rest % a.tiles_per_row), seq = (int)(rest / a.tiles_per_row);
+        const int64_t row = (int64_t)seq * RPS0 + rr;
+        const int32_t *line =
+            lane == 0 ? c.row_len + row
+                      : (lane == 1 ? c.block_table + row * c.max_pages_per_row + min(t * kPagesPerTile, c.max_pages_per_row - 1)
+                                   : a.q.num_q + seq);
+        if (lane < 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
+        const int32_t *sp = c.slot_pos + row * c.max_slots + (int64_t)t * kTileKeys;
+        const int nk = (int)min((int64_t)kTileKeys, c.max_slots - (int64_t)t * kTileKeys);
+        if (lane * 32 < nk) asm volatile("prefetch.global.L2 [%0];" ::"l"(sp + lane * 32));
+        const int32_t *qp = a.q.q_pos + (int64_t)seq * a.q.max_q;
+        for (int j = lane * 32; j < a.q.max_q; j += 32 * 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(qp + j));
+    }
     // zero the operand buffers once so rows no load ever fills hold finite values
     for (int i = threadIdx.x; i < (2 * PL::kABytes + PL::kStages * PL::kBBytes) / 16; i += kThreads)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
@@ -363,11 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int k = 0; k < kMeta; ++k) {
             mbar_init(&ctl.m_full[k], 1);
-            mbar_init(&ctl.m_empty[k], 1 + kEpiWarps);
+            mbar_init(&ctl.m_empty[k], kEpiWarps);
         }
         for (int k = 0; k < kTiles; ++k) {
             mbar_init(&ctl.t_full[k], 1);
-            mbar_init(&ctl.t_empty[k], 1);
+            mbar_init(&ctl.t_empty[k], 2);  // TMA and MMA warps
         }
         mbar_init(&ctl.drain, 1);
         ctl.abort = 0;
@@ -812,49 +833,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");  // no copy into shared memory outlives the CTA
     } else if (warp == 1) {
         // ============================== MMA issuer ==============================
-        uint32_t qs = 0, qph = 0, mk = 0, mph = 0, ab = 0, abph = 0;
-        uint32_t tm = 0;  // K tiles consumed so far (same order as the producer's loads)
+        // Follows the tile ring like the TMA warp: per tile the K buffer, per visible block the Q stage and an
+        // accumulator buffer; two M=128 x N=128 x K=D products per block, one thread issuing.
+        uint32_t qs = 0, qph = 0, tk = 0, tph = 0, ab = 0, abph = 0;
+        uint32_t tm = 0;  // K tiles consumed so far (same order as the TMA warp's loads)
         bool issued = false;
+        const uint32_t a_lo0 = desc_lo(smem_u32(sA)), b_lo0 = desc_lo(smem_u32(sB));
         for (;;) {
-            if (!mbar_wait(&ctl.m_full[mk], mph, ctl, a.status, -1)) break;
-            const Item &it = items[mk];
-            const int row = it.row;
+            if (!mbar_wait(&ctl.t_full[tk], tph, ctl, a.status, -1)) break;
+            const TileRec &R = ctl.trec[tk];
+            const int row = R.row;
             if (row < 0) break;
-            const int blk = it.blk, flags = it.flags;
-            if (blk >= 0) {
-                const uint32_t abuf = tm & 1;
-                if (flags & kFirst) {
-                    if (!mbar_wait(&ctl.a_full[abuf], (tm >> 1) & 1, ctl, a.status, row)) break;
-                }
-                if (!mbar_wait(&ctl.q_full[qs], qph, ctl, a.status, row)) break;
-                if (!mbar_wait(&ctl.acc_empty[ab], abph ^ 1, ctl, a.status, row)) break;
+            const uint32_t abuf = tm & 1;
+            if (!mbar_wait(&ctl.a_full[abuf], (tm >> 1) & 1, ctl, a.status, row)) break;
+            const uint32_t a_lo = a_lo0 + ((abuf * PL::kABytes) >> 4);
+            bool ok = true;
+            for (int b = R.first_vis; b >= 0;) {
+                const int bn = next_visible(R.vmask, b);
+                if (!mbar_wait(&ctl.q_full[qs], qph, ctl, a.status, row)) { ok = false; break; }
+                if (!mbar_wait(&ctl.acc_empty[ab], abph ^ 1, ctl, a.status, row)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
+                    const uint32_t b_lo = b_lo0 + ((qs * PL::kBBytes) >> 4);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t d = tmem + ab * 256 + h * kCols;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const int kc = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ad = sw128_desc(
-                                smem_u32(sA + abuf * PL::kABytes + kc * (kTileKeys * 128) + h * (128 * 128) + ko));
-                            const uint64_t bd = sw128_desc(smem_u32(sB + qs * PL::kBBytes + kc * (kCols * 128) + ko));
-                            mma_bf16(d, ad, bd, kk > 0 ? 1u : 0u);
+                            const uint32_t ao = (uint32_t)(((kk >> 2) * (kTileKeys * 128) + h * (128 * 128) + (kk & 3) * 32) >> 4);
+                            const uint32_t bo = (uint32_t)(((kk >> 2) * (kCols * 128) + (kk & 3) * 32) >> 4);
+                            if (kk == 0)
+                                mma_bf16<false>(d, a_lo + ao, b_lo + bo);
+                            else
+                                mma_bf16<true>(d, a_lo + ao, b_lo + bo);
                         }
                     }
                     mma_commit(&ctl.q_empty[qs]);
                     mma_commit(&ctl.acc_full[ab]);
-                    if (flags & kLast) mma_commit(&ctl.a_empty[abuf]);
+                    if (bn < 0) mma_commit(&ctl.a_empty[abuf]);
                 }
                 issued = true;
-                if (flags & kLast) ++tm;
                 __syncwarp();
                 if (++qs == PL::kStages) { qs = 0; qph ^= 1; }
                 if (++ab == 2) { ab = 0; abph ^= 1; }
+                b = bn;
             }
+            if (!ok) break;
+            ++tm;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl.m_empty[mk]);
-            if (++mk == kMeta) { mk = 0; mph ^= 1; }
+            if (lane == 0) mbar_arrive(&ctl.t_empty[tk]);
+            if (++tk == kTiles) { tk = 0; tph ^= 1; }
         }
         // all MMAs issued by this thread are complete before TMEM is released
         if (issued) {
