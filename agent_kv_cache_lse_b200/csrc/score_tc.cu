@@ -27,11 +27,11 @@
 //              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) into one of two TMEM
 //              accumulator buffers (4 x 128 of the 512 columns).
 //   warps 3-18 epilogue: (TMEM lane quadrant, key half, column half); thread = key;
-//              tcgen05.ld 16 columns at a time (double-buffered), x = acc * log2e/sqrt(D) - lse_col * log2e
-//              in packed f32x2 arithmetic, causal select, 2^x (half on the MUFU unit,
-//              half by polynomial on the FMA pipes), sums in registers.  The two column
-//              halves of a key are added through shared memory at the end of the tile;
-//              one coalesced store per key per tile.
+//              tcgen05.ld 16 columns at a time (double-buffered), x = acc * log2e/sqrt(D)
+//              - lse_col * log2e in packed f32x2 arithmetic, causal select, 2^x (three
+//              quarters on the MUFU unit, a quarter by polynomial on the FMA pipes), sums in
+//              registers.  The two column halves of a key are added through shared memory
+//              at the end of the tile; one coalesced store per key per tile.
 // Blocks whose queries all precede the tile's first key are skipped entirely
 // (no load, no MMA, no epilogue work).  Every barrier wait is bounded (about one
 // second of global time); on expiry the kernel records KVC_DEV_TIMEOUT, drains its
@@ -268,9 +268,9 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 
 // Sixteen columns of a key's accumulator row: x = acc * log2(e)/sqrt(D) - lse_col * log2(e), causal select
 // (unless every column of the block sees every key of the warp), 2^x, running sums.  Columns go in pairs
-// through packed f32x2 arithmetic; in each group of four, two exponentials run on the MUFU unit and two on
-// the FMA pipes.  An absent column has -lse = -inf: it adds 0 (MUFU) or 2^-126 (polynomial), both far below
-// any tolerance.
+// through packed f32x2 arithmetic; of every eight exponentials, six run on the MUFU unit and two on the FMA
+// pipes (the MUFU unit is the scarcer resource, issue slots the next one).  An absent column has
+// -lse = -inf: it adds 0 (MUFU) or 2^-126 (polynomial), both far below any tolerance.
 __device__ __forceinline__ void epi16(const uint32_t (&r)[16], const float *nL, const int32_t *qp, int kpos, float sc,
                                       bool fast, float2 &am, float2 &ap) {
     const float4 *L4 = reinterpret_cast<const float4 *>(nL);
@@ -284,7 +284,7 @@ __device__ __forceinline__ void epi16(const uint32_t (&r)[16], const float *nL, 
             const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])),
                                           sc2, make_float2(l.z, l.w));
             am = __fadd2_rn(am, make_float2(ex2(x01.x), ex2(x01.y)));
-            ap = __fadd2_rn(ap, exp2_fma2(x23));
+            ap = __fadd2_rn(ap, (c4 & 1) ? exp2_fma2(x23) : make_float2(ex2(x23.x), ex2(x23.y)));
         }
     } else {
         const int4 *P4 = reinterpret_cast<const int4 *>(qp);
@@ -301,7 +301,7 @@ __device__ __forceinline__ void epi16(const uint32_t (&r)[16], const float *nL, 
             x23.x = p.z >= kpos ? x23.x : -INFINITY;
             x23.y = p.w >= kpos ? x23.y : -INFINITY;
             am = __fadd2_rn(am, make_float2(ex2(x01.x), ex2(x01.y)));
-            ap = __fadd2_rn(ap, exp2_fma2(x23));
+            ap = __fadd2_rn(ap, (c4 & 1) ? exp2_fma2(x23) : make_float2(ex2(x23.x), ex2(x23.y)));
         }
     }
 }
