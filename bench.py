@@ -15,6 +15,7 @@ the path shards by sequence and needs no collective).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -283,7 +284,8 @@ def run_ours(args, rank, world, device):
                    "queries": int(queries.num_q.sum()), "budget": spec.budget, "seq_len": 32768,
                    "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before every step"},
         "roofline": {"kernel": "score_tc_kernel (kvc_score_from_lse)", "bound": "tensor", "achieved": achieved,
-                     "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst, "traffic": None,
+                     "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst, "traffic": profiled_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{peak_kind} bf16 dense (burst)", "flops_per_launch": work["flops"],
                      "ms_per_launch": score_avg,
                      "exp_rate_per_s": work["exps"] / (score_avg / 1e3),
@@ -302,6 +304,28 @@ def run_ours(args, rank, world, device):
 
 
 EvictionRound_KERNELS = 8
+
+SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
+
+
+def profiled_traffic():
+    """DRAM bytes per score_tc_kernel launch from the committed ncu summary, or None when the kernel source
+    has changed since those counters were taken (the summary records the source's sha256)."""
+    try:
+        fields = {}
+        with open(SCORE_PROFILE) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, _, v = line.partition(":")
+                    fields[k.strip()] = v.strip()
+        src = os.path.join(ROOT, fields["source"])
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if digest != fields["source_sha256"]:
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def run_e2e(args, spec, cache, queries, logits, rnd, pristine, device):

@@ -104,3 +104,19 @@ def test_layout_block_tables_are_disjoint():
     assert used.max() < lay.num_pages
     for r in range(spec.rows):
         assert (bt[r] >= 0).sum() == -(-int(lay.row_len[r]) // 16)
+
+
+def test_bench_traffic_follows_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while the kernel source hash matches."""
+    import hashlib
+    import bench
+    t = bench.profiled_traffic()
+    assert t is None or t > 0
+    src = tmp_path / "k.cu"
+    src.write_text("x")
+    prof = tmp_path / "p.md"
+    prof.write_text(f"source: {src}\nsource_sha256: {'0' * 64}\ndram_bytes_per_launch: 5\n")
+    monkeypatch.setattr(bench, "SCORE_PROFILE", str(prof))
+    assert bench.profiled_traffic() is None
+    prof.write_text(f"source: {src}\nsource_sha256: {hashlib.sha256(b'x').hexdigest()}\ndram_bytes_per_launch: 5\n")
+    assert bench.profiled_traffic() == 5
