@@ -259,7 +259,7 @@ kvc_status kvc_confidence_ratchet(const float *logits, int32_t num_seqs, int32_t
     if (num_seqs <= 0 || num_seqs > 65535) return fail(KVC_ERR_INVALID_ARGUMENT, "num_seqs out of range");
     if (steps < 0 || steps > params->max_steps || steps > 65535)
         return fail(KVC_ERR_INVALID_ARGUMENT, "steps must be in [0, params->max_steps]");
-    if (vocab <= 0 || vocab > 8 * 40960) return fail(KVC_ERR_UNSUPPORTED, "vocab must be in [1, 327680]");
+    if (vocab <= 0 || vocab > (1 << 24)) return fail(KVC_ERR_UNSUPPORTED, "vocab must be in [1, 2^24]");
     return cuda_status(kvc::launch_ratchet(logits, num_seqs, steps, vocab, state, budget, confidence_out, *params,
                                            d_status, (cudaStream_t)stream),
                        "kvc_confidence_ratchet launch");

@@ -27,12 +27,15 @@ struct LrfuArgs {
     int binary;
     int32_t *status;
     int slice_cap;    // scores cached in shared memory when a CTA's slice fits
+    int weight_cap;   // fixed-point masses cached too when the slice fits this
 };
 
 __global__ void __launch_bounds__(kThreads, 1) lrfu_kernel(LrfuArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RowShared &sh = *reinterpret_cast<RowShared *>(smem_raw);
     uint32_t *kc = reinterpret_cast<uint32_t *>(smem_raw + sizeof(RowShared));
+    unsigned long long *qw = reinterpret_cast<unsigned long long *>(
+        smem_raw + sizeof(RowShared) + (((size_t)a.slice_cap * 4 + 15) & ~(size_t)15));
     RowCtx rc = row_ctx();
     const int row = blockIdx.x / rc.nranks;
     const CacheView &c = a.c;
@@ -47,6 +50,7 @@ __global__ void __launch_bounds__(kThreads, 1) lrfu_kernel(LrfuArgs a) {
     float *crf = a.crf + (int64_t)row * c.max_slots;
     const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots;
     const bool cached = per <= a.slice_cap;
+    const bool wcached = cached && per <= a.weight_cap;
 
     // stage the slice (raw fp32 bits, sign cleared so -0.0 ranks as 0), validate, row maximum
     int bad = 0;
@@ -89,12 +93,17 @@ __global__ void __launch_bounds__(kThreads, 1) lrfu_kernel(LrfuArgs a) {
         const int e = 48 - E;
         auto q = [&](int i) -> unsigned long long { return (unsigned long long)ldexp((double)sval(i), e); };
         unsigned long long part = 0;
-        for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) part += q(i);
-        const unsigned long long Sq = row_sum_u64(rc, sh, part);
+        for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+            const unsigned long long w = q(i);
+            part += w;
+            if (wcached) qw[i - lo] = w;  // each pass of the search below reads it instead of recomputing
+        }
+        const unsigned long long Sq = row_sum_u64(rc, sh, part);  // its cluster barrier also orders qw
+        auto qv = [&](int i) -> unsigned long long { return wcached ? qw[i - lo] : q(i); };
         unsigned long long target = (unsigned long long)ceil((double)a.hit_mass * (double)Sq);
         if (target > Sq) target = Sq;
         if (target >= 1) {
-            const RadixResult r = row_radix_desc<true>(rc, sh, lo, hi, target, skey, q,
+            const RadixResult r = row_radix_desc<true>(rc, sh, lo, hi, target, skey, qv,
                                                        [&](int i) { return skey(i) != 0u; });
             T = r.key;
             const unsigned long long qT = (unsigned long long)ldexp((double)__uint_as_float(T), e);
@@ -166,10 +175,11 @@ cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, flo
     if ((c.max_slots + C - 1) / C > 65536) return cudaErrorInvalidValue;
     const int per = (int)((c.max_slots + C - 1) / C);
     const int cap = per < 40960 ? per : 0;
-    const size_t smem = sizeof(RowShared) + (size_t)cap * 4;
+    const int wcap = cap > 0 && per <= 12288 ? per : 0;
+    const size_t smem = sizeof(RowShared) + (((size_t)cap * 4 + 15) & ~(size_t)15) + (size_t)wcap * 8;
     cudaError_t e = cudaFuncSetAttribute(lrfu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    LrfuArgs a{c, scores, crf, decay, hit_mass, binary ? 1 : 0, status, cap};
+    LrfuArgs a{c, scores, crf, decay, hit_mass, binary ? 1 : 0, status, cap, wcap};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(c.rows * C));
     cfg.blockDim = dim3(kThreads);

@@ -8,14 +8,15 @@
 // small and grows it by 1.75x (initial 512, cap 30,000); it never shrinks.
 //
 // Launch A (confidence): a cluster of kCluster CTAs per (sequence, step) row of
-//   logits.  Each CTA stages its slice of the vocabulary in shared memory, reduces
-//   its (max, sum of exp) and its exact top-k list, and the leader CTA merges the
-//   cluster's partials through distributed shared memory into c_t.  The slice arrives
-//   by bulk (TMA) copies when the row is 16-byte aligned.  The local top-k takes the
-//   k-th largest of the warps' top-2 per-thread maxima as a lower bound, collects the
-//   values above it (a few dozen) and sorts them with a warp bitonic network; when
-//   more than 64 qualify (many equal logits) it falls back to an exact radix search
-//   over the staged slice.
+//   logits, each CTA a slice of the vocabulary, read straight from global memory with
+//   16-byte loads (no staging: the logits of a round do not fit in the shared memory of
+//   the GPU, so staging would need a second wave of CTAs).  Pass 1 keeps a running
+//   (max, sum of exp) per thread; the k-th largest of the warps' top-4 per-thread
+//   maxima is a lower bound for the slice's k-th largest logit.  Pass 2 re-reads the
+//   slice (from L2) for the values at or above that bound (a few dozen), which a warp
+//   bitonic network sorts; when more than 64 qualify (many equal logits) an exact radix
+//   search over the slice takes over.  The leader CTA merges the cluster's (max, sum)
+//   pairs and sorted top-k lists through distributed shared memory into c_t.
 // Launch B (ratchet): one warp per sequence pools the newly completed windows,
 //   updates the least-squares sums, evaluates the fit once and moves the budget.
 #include <cooperative_groups.h>
@@ -31,7 +32,8 @@ namespace kvc {
 namespace {
 
 constexpr int kCluster = 8;
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTopK = 64;
 
 size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -52,14 +54,12 @@ struct ConfArgs {
     const float *logits;
     int32_t steps, vocab, chunk;
     int32_t top_k;
-    int32_t bulk;       // rows and slices 16-byte aligned: stage with bulk copies
+    int32_t vec;        // rows and slices 16-byte aligned: 16-byte loads
     float *hist;        // [seqs][hist_len]
     int32_t hist_len, window;
     float *conf_out;    // [seqs][steps] or null
     int32_t *status;
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 // 2^x by the MUFU unit (ex2.approx, relative error ~2^-22): ample for the log-sum-exp of a step.
 __device__ __forceinline__ float exp2f_fast(float x) {
@@ -94,22 +94,40 @@ __device__ __forceinline__ void warp_sort64_desc(float &a, float &b) {
 }
 
 struct ConfShared {
-    RadixShared rs;
     float cand[64];
-    float topk[kMaxTopK];
-    float wtop[32];      // top-2 per warp of the per-thread maxima
+    float topk[kMaxTopK];        // this CTA's top-k, descending (-inf pads a short slice)
+    float wtop[32];              // top-4 per warp of the per-thread maxima
     float red_f[32];
     double red_d[32];
     int red_i[32];
-    uint64_t bar;
+    unsigned int hist[256];      // exact fallback: digit counts
+    uint32_t fb_prefix, fb_pmask;
+    int fb_above, fb_remaining;
     float cmax;
     double csum;
     int ncand;
     int nbad;
 };
 
+// Running (max m, sum s of exp(z - m)) of a thread: one exponential per value, two when the max moves.
+struct RunLse {
+    float m = -INFINITY, s = 0.f;
+    int bad = 0;
+    __device__ __forceinline__ void add(float z) {
+        if (!is_finite(z)) {
+            if (z != -INFINITY) bad = 1;  // -inf contributes nothing; NaN and +inf are errors
+            return;
+        }
+        if (z > m) {
+            s = s * exp2f_fast((m - z) * 1.4426950408889634f) + 1.f;
+            m = z;
+        } else {
+            s += exp2f_fast((z - m) * 1.4426950408889634f);
+        }
+    }
+};
+
 __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
-    extern __shared__ __align__(16) float zs[];
     __shared__ ConfShared sh;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -118,75 +136,52 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
     const float *row = a.logits + ((int64_t)seq * a.steps + step) * a.vocab;
     const int lo = min(a.vocab, rank * a.chunk), hi = min(a.vocab, lo + a.chunk);
     const int cnt = hi - lo;
+    const float *z = row + lo;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) sh.ncand = 0;
+    // the slice as 16-byte vectors (a.vec: the slice starts 16-byte aligned) plus a scalar tail
+    const int n4 = a.vec ? cnt >> 2 : 0;
+    const float4 *z4 = reinterpret_cast<const float4 *>(z);
 
-    // stage the slice in shared memory: one bulk copy when the row slice is 16-byte aligned
-    if (tid == 0) {
-        sh.ncand = 0;
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&sh.bar)) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    const bool bulk = a.bulk && cnt > 0;
-    if (bulk) {
-        if (tid == 0) {
-            const uint32_t bytes = (uint32_t)cnt * 4u;
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&sh.bar)), "r"(bytes)
-                         : "memory");
-            for (uint32_t off = 0; off < bytes; off += 16384u) {
-                const uint32_t sz = min(16384u, bytes - off);
-                asm volatile(
-                    "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                        smem_addr(zs) + off),
-                    "l"(reinterpret_cast<const char *>(row + lo) + off), "r"(sz), "r"(smem_addr(&sh.bar))
-                    : "memory");
-            }
+    // pass 1: running (max, sum of exp) per thread, four vectors in flight
+    RunLse r;
+    for (int i = tid; i < n4; i += 4 * kThreads) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = i + u * kThreads < n4 ? z4[i + u * kThreads] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            r.add(v[u].x);
+            r.add(v[u].y);
+            r.add(v[u].z);
+            r.add(v[u].w);
         }
-        // bounded wait for the copy (a second at most)
-        uint32_t done = 0;
-        long long t0 = clock64();
-        while (!done) {
-            asm volatile(
-                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-                : "=r"(done)
-                : "r"(smem_addr(&sh.bar))
-                : "memory");
-            if (!done && clock64() - t0 > (1ll << 31)) {
-                if (tid == 0) report(a.status, KVC_DEV_TIMEOUT, seq);
-                break;
-            }
-        }
-    } else {
-        for (int i = tid; i < cnt; i += kThreads) zs[i] = row[lo + i];
-        __syncthreads();
     }
-    // per-thread maximum and finiteness (from shared memory)
-    float tmax = -INFINITY;
-    int bad = 0;
-    for (int i = tid; i < cnt; i += kThreads) {
-        const float z = zs[i];
-        bad |= !is_finite(z);
-        tmax = fmaxf(tmax, z);
-    }
-    // lower bound tau0 for the slice's k-th largest: the k-th largest of the 32 warp top-2 values
+    for (int i = 4 * n4 + tid; i < cnt; i += kThreads) r.add(z[i]);
+    const float tmax = r.m;
+
+    // lower bound tau0 for the slice's k-th largest: the k-th largest of the warps' top-4 per-thread maxima
+    // (32 distinct values of the slice)
     {
-        float m1 = tmax;
+        float cur = tmax;
+        bool taken = false;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-        const unsigned who = __ballot_sync(0xffffffffu, tmax == m1);
-        float m2 = (lane == __ffs(who) - 1) ? -INFINITY : tmax;
+        for (int q = 0; q < 4; ++q) {
+            float mq = taken ? -INFINITY : cur;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-        if (lane == 0) {
-            sh.wtop[2 * warp] = m1;
-            sh.wtop[2 * warp + 1] = m2;
+            for (int o = 16; o > 0; o >>= 1) mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+            const unsigned who = __ballot_sync(0xffffffffu, !taken && cur == mq);
+            if (lane == __ffs(who) - 1) taken = true;
+            if (lane == 0) sh.wtop[4 * warp + q] = mq;
         }
     }
-    const float cmax = block_max(tmax, sh.red_f);   // also orders the wtop writes
-    bad = block_or(bad, sh.red_i);
+    const float cmax = block_max(tmax, sh.red_f);  // also orders the wtop writes
+    const double csum = block_sum<double>(cmax == -INFINITY ? 0.0 : (double)r.s * exp((double)r.m - (double)cmax),
+                                          sh.red_d);
+    const int bad = block_or(r.bad, sh.red_i);
     float tau0 = -INFINITY;
-    if (cnt >= K && K <= 2 * (kThreads / 32)) {
-        // every thread ranks the 32 candidates for the bound; identical in all threads
+    if (cnt >= K && K <= 4 * kWarps) {
+        // every warp ranks the 32 values for the bound; identical in all threads
         const float v = sh.wtop[lane];
         int above = 0;
         for (int f = 0; f < 32; ++f) {
@@ -196,19 +191,29 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
         const unsigned is_k = __ballot_sync(0xffffffffu, above == K - 1);
         tau0 = __shfl_sync(0xffffffffu, v, __ffs(is_k) - 1);
     }
-    // log-sum-exp partial and candidates z >= tau0 (one pass over shared memory)
-    float part = 0.f;
+    // pass 2 (the slice is in L2 now): candidates z >= tau0
+    auto cand = [&](float x) {
+        if (x >= tau0 && x != -INFINITY) {
+            const int at = atomicAdd(&sh.ncand, 1);
+            if (at < 64) sh.cand[at] = x;
+        }
+    };
     if (cmax != -INFINITY) {
-        for (int i = tid; i < cnt; i += kThreads) {
-            const float z = zs[i];
-            part += exp2f_fast((z - cmax) * 1.4426950408889634f);
-            if (z >= tau0) {
-                const int at = atomicAdd(&sh.ncand, 1);
-                if (at < 64) sh.cand[at] = z;
+        for (int i = tid; i < n4; i += 4 * kThreads) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = i + u * kThreads < n4 ? z4[i + u * kThreads] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                cand(v[u].x);
+                cand(v[u].y);
+                cand(v[u].z);
+                cand(v[u].w);
             }
         }
+        for (int i = 4 * n4 + tid; i < cnt; i += kThreads) cand(z[i]);
     }
-    const double csum = block_sum<double>((double)part, sh.red_d);  // also orders the candidate writes
+    __syncthreads();
     const int ncand = sh.ncand;
     if (ncand <= 64) {
         if (warp == 0) {
@@ -219,17 +224,59 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
             if (lane + 32 < K) sh.topk[lane + 32] = y;
         }
     } else {
-        // exact fallback (many equal logits): k-th largest key over the staged slice, then values above it
-        const RadixResult r = radix_search_desc<false>(
-            cnt, (unsigned long long)K, [&](int i) { return float_key(zs[i]); }, [](int) { return 1ull; },
-            [](int) { return true; }, sh.rs);
-        const float T = key_float(r.key);
+        // exact fallback (many equal logits): radix search for the k-th largest key of the slice (four 8-bit
+        // digits, counts in shared memory), then the values above it, sorted, then copies of it
+        if (tid == 0) {
+            sh.fb_prefix = 0;
+            sh.fb_pmask = 0;
+            sh.fb_above = 0;
+            sh.fb_remaining = K;
+        }
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0;
+            __syncthreads();
+            const uint32_t prefix = sh.fb_prefix, pmask = sh.fb_pmask;
+            for (int i = tid; i < cnt; i += kThreads) {
+                const float x = z[i];
+                if (x == -INFINITY || !is_finite(x)) continue;
+                const uint32_t k = float_key(x);
+                if ((k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int run = 0;
+                for (int b = 255; b >= 0; --b) {
+                    const int c = (int)sh.hist[b];
+                    if (run + c >= sh.fb_remaining) {
+                        sh.fb_above += run;
+                        sh.fb_remaining -= run;
+                        sh.fb_prefix |= (uint32_t)b << shift;
+                        sh.fb_pmask |= 255u << shift;
+                        break;
+                    }
+                    run += c;
+                }
+            }
+            __syncthreads();
+        }
+        const uint32_t T = sh.fb_prefix;
+        const int above = sh.fb_above;  // values strictly greater than T: fewer than k
         if (tid == 0) sh.ncand = 0;
         __syncthreads();
-        for (int i = tid; i < cnt; i += kThreads)
-            if (float_key(zs[i]) > r.key) sh.topk[atomicAdd(&sh.ncand, 1)] = zs[i];
+        for (int i = tid; i < cnt; i += kThreads) {
+            const float x = z[i];
+            if (x != -INFINITY && is_finite(x) && float_key(x) > T) sh.cand[atomicAdd(&sh.ncand, 1)] = x;
+        }
         __syncthreads();
-        for (int t = (int)r.above + tid; t < K; t += kThreads) sh.topk[t] = T;
+        if (warp == 0) {
+            float x = lane < above ? sh.cand[lane] : -INFINITY;
+            float y = lane + 32 < above ? sh.cand[lane + 32] : -INFINITY;
+            warp_sort64_desc(x, y);
+            const float tv = key_float(T);
+            if (lane < K) sh.topk[lane] = lane < above ? x : tv;
+            if (lane + 32 < K) sh.topk[lane + 32] = lane + 32 < above ? y : tv;
+        }
     }
     if (tid == 0) {
         sh.cmax = cmax;
@@ -238,7 +285,7 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
     }
     cluster.sync();
     if (rank == 0) {
-        // merge the cluster: LSE from the partial (max, sum) pairs; global top-k from the local lists
+        // merge the cluster: LSE from the (max, sum) pairs; the sum of the k largest from the sorted lists
         __shared__ float allv[kCluster * kMaxTopK];
         __shared__ float pm[kCluster];
         __shared__ double ps[kCluster];
@@ -247,38 +294,39 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
             ConfShared *peer = cluster.map_shared_rank(&sh, tid);
             pm[tid] = peer->cmax;
             ps[tid] = peer->csum;
+            if (tid == 0) anybad = 0;
         }
-        if (tid == 0) anybad = 0;
+        for (int e = tid; e < kCluster * K; e += kThreads) allv[e] = cluster.map_shared_rank(&sh, e / K)->topk[e % K];
         __syncthreads();
-        for (int e = tid; e < kCluster * K; e += kThreads) {
-            ConfShared *peer = cluster.map_shared_rank(&sh, e / K);
-            allv[e] = peer->topk[e % K];
-            if (e % K == 0 && peer->nbad) atomicOr(&anybad, 1);
-        }
-        __syncthreads();
-        double contrib = 0.0;
-        for (int e = tid; e < kCluster * K; e += kThreads) {
-            const float v = allv[e];
-            int above = 0;
-            for (int f = 0; f < kCluster * K; ++f) {
-                const float w = allv[f];
-                above += (w > v) || (w == v && f < e);
+        if (tid < kCluster && cluster.map_shared_rank(&sh, tid)->nbad) atomicOr(&anybad, 1);
+        if (warp == 0) {
+            // k steps of taking the largest head among the kCluster lists (lane r holds list r's head)
+            int head = 0;
+            double topsum = 0.0;
+            for (int t = 0; t < K; ++t) {
+                const float hv = (lane < kCluster && head < K) ? allv[lane * K + head] : -INFINITY;
+                float best = hv;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+                if (best == -INFINITY) break;  // fewer than k values in the whole row
+                const unsigned who = __ballot_sync(0xffffffffu, lane < kCluster && hv == best);
+                if (lane == __ffs(who) - 1) ++head;
+                topsum += (double)best;
             }
-            if (above < K && v != -INFINITY) contrib += (double)v;
-        }
-        const double topsum = block_sum<double>(contrib, sh.red_d);
-        if (tid == 0) {
-            float M = -INFINITY;
-            for (int r = 0; r < kCluster; ++r) M = fmaxf(M, pm[r]);
-            double S = 0.0;
-            for (int r = 0; r < kCluster; ++r)
-                if (pm[r] != -INFINITY) S += ps[r] * exp((double)pm[r] - (double)M);
-            const double lse = (double)M + log(S);
-            const int kk = min(K, a.vocab);
-            const double c = lse - topsum / kk;
-            if (anybad) report(a.status, KVC_DEV_NONFINITE, seq);
-            a.hist[(int64_t)seq * a.hist_len + (a.window - 1) + step] = (float)c;
-            if (a.conf_out) a.conf_out[(int64_t)seq * a.steps + step] = (float)c;
+            __syncwarp();
+            if (lane == 0) {
+                float M = -INFINITY;
+                for (int q = 0; q < kCluster; ++q) M = fmaxf(M, pm[q]);
+                double S = 0.0;
+                for (int q = 0; q < kCluster; ++q)
+                    if (pm[q] != -INFINITY) S += ps[q] * exp((double)pm[q] - (double)M);
+                const double lse = (double)M + log(S);
+                const int kk = min(K, a.vocab);
+                const double c = lse - topsum / kk;
+                if (anybad) report(a.status, KVC_DEV_NONFINITE, seq);
+                a.hist[(int64_t)seq * a.hist_len + (a.window - 1) + step] = (float)c;
+                if (a.conf_out) a.conf_out[(int64_t)seq * a.steps + step] = (float)c;
+            }
         }
     }
     cluster.sync();
@@ -397,15 +445,12 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
     float *hist = reinterpret_cast<float *>(static_cast<char *>(state) + l.state_bytes);
     if (steps > 0) {
         const int chunk = ((vocab + kCluster - 1) / kCluster + 3) / 4 * 4;  // whole 16-byte units per slice
-        const size_t smem = (size_t)chunk * sizeof(float);
-        cudaError_t e = cudaFuncSetAttribute(confidence_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        const int bulk = (vocab % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
-        ConfArgs a{logits, steps, vocab, chunk, p.top_k, bulk, hist, l.hist_len, p.window, conf_out, status};
+        const int vec = (vocab % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
+        ConfArgs a{logits, steps, vocab, chunk, p.top_k, vec, hist, l.hist_len, p.window, conf_out, status};
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(kCluster, (unsigned)steps, (unsigned)num_seqs);
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = 0;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -414,7 +459,7 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, confidence_kernel, a);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, confidence_kernel, a);
         if (e != cudaSuccess) return e;
     }
     UpdArgs u{st, hist, budget, num_seqs, steps, l.hist_len, p};
@@ -422,7 +467,5 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
     return cudaGetLastError();
 }
 
-int ratchet_max_top_k() { return kMaxTopK; }
-int ratchet_max_vocab() { return 40960 * kCluster; }
 
 }  // namespace kvc

@@ -151,16 +151,18 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
         sh.remaining = target;
         sh.eq_count = 0;
     }
+    auto zero_hist = [&](RowHist &z) {
+        for (int i = tid; i < kRowBins; i += blockDim.x) {
+            z.cnt[i] = 0;
+            if (kMass) z.wt[0][i] = z.wt[1][i] = z.wt[2][i] = 0;
+        }
+    };
+    zero_hist(sh.hist[rc.par & 1]);
     __syncthreads();
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         const int b = rc.par & 1;
         RowHist &h = sh.hist[b];
-        for (int i = tid; i < kRowBins; i += blockDim.x) {
-            h.cnt[i] = 0;
-            if (kMass) h.wt[0][i] = h.wt[1][i] = h.wt[2][i] = 0;
-        }
-        __syncthreads();
         const uint32_t prefix = sh.prefix, pmask = sh.pmask;
         const int span = hi - lo;
         const int nround = (span + blockDim.x - 1) / blockDim.x * blockDim.x;
@@ -210,6 +212,8 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
             }
         }
         rc.cl.sync();
+        // the other buffer was last read by the peers before this barrier: clear it for the next pass now
+        if (pass < 3) zero_hist(sh.hist[b ^ 1]);
         for (int i = tid; i < kRowBins; i += blockDim.x) {
             unsigned int c = 0;
             unsigned long long w = 0;

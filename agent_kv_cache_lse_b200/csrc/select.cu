@@ -69,9 +69,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
             }
         }
     }
-    float dummy = 0.f;
-    row_max_or(rc, sh, dummy, bad);
-    if (bad) {
+    // one collective: the protected count and whether any CRF is not finite
+    int tot[2], below[2];
+    row_sum_int2(rc, sh, nprot, bad, tot, below);
+    if (tot[1] != 0) {
         // keep everything on a faulted row: nothing is evicted
         for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) keep[i] = 1;
         if (rc.rank == 0 && threadIdx.x == 0) {
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         rc.cl.sync();
         return;
     }
-    nprot = row_sum_int(rc, sh, nprot, nullptr);
+    nprot = tot[0];
     auto key = [&](int i) -> uint32_t {
         if (cached) return kc[i - lo];
         const float v = crf[i];

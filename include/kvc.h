@@ -279,8 +279,8 @@ kvc_status kvc_ratchet_init(void *state, int32_t *budget, int32_t num_seqs,
  * line y = a + b*j.  After the round, if at least min_points points are in the fit and
  * b < 0, budget <- min(floor(budget * grow_num / grow_den), cap), the fit restarts, and
  * the expansion step is recorded.  The budget never shrinks.
- * logits: [num_seqs][steps][vocab] fp32.  budget: [num_seqs] int32 (written).
- * confidence_out: [num_seqs][steps] fp32 c_t, or NULL.
+ * logits: [num_seqs][steps][vocab] fp32, vocab in [1, 2^24] (else KVC_ERR_UNSUPPORTED).
+ * budget: [num_seqs] int32 (written).  confidence_out: [num_seqs][steps] fp32 c_t, or NULL.
  */
 kvc_status kvc_confidence_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab,
                                   void *state, int32_t *budget, float *confidence_out,
