@@ -278,7 +278,8 @@ def run_ours(args, rank, world, device):
     exp_ceiling = 16 * 148 * sm_mhz * 1e6
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "ms_per_step": ms_step, "ms_per_step_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator; shapes of the agent-trace workload)",
         "config": {"workload": WORKLOAD, "entries_per_step": work["entries"], "rows": spec.rows,
                    "queries": int(queries.num_q.sum()), "budget": spec.budget, "seq_len": 32768,
