@@ -237,6 +237,26 @@ size_t kvc_ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params *param
     return kvc::ratchet_state_bytes(num_seqs, *params);
 }
 
+kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_seqs, int32_t num_layers,
+                             int32_t num_q_heads, int32_t head_dim, int32_t max_q, kvc_dtype dtype, float *beacons,
+                             int32_t *counts, int32_t num_beacons, void *beacon_q, int32_t out_max_q,
+                             int32_t *d_status, kvc_stream_t stream) {
+    g_err[0] = 0;
+    if (!q || !num_q || !beacons || !counts) return fail(KVC_ERR_INVALID_ARGUMENT, "q, num_q, beacons and counts are required");
+    if (dtype != KVC_BF16 && dtype != KVC_F32) return fail(KVC_ERR_UNSUPPORTED, "dtype must be bf16 or f32");
+    if (num_seqs <= 0 || num_layers <= 0 || num_q_heads <= 0)
+        return fail(KVC_ERR_INVALID_ARGUMENT, "num_seqs, num_layers and num_q_heads must be positive");
+    if ((int64_t)num_seqs * num_layers * num_q_heads > INT32_MAX) return fail(KVC_ERR_UNSUPPORTED, "too many groups");
+    if (head_dim <= 0 || head_dim > 256) return fail(KVC_ERR_UNSUPPORTED, "head_dim must be in [1, 256]");
+    if (num_beacons <= 0 || num_beacons > 64) return fail(KVC_ERR_UNSUPPORTED, "num_beacons must be in [1, 64]");
+    if (max_q <= 0 || max_q > 65536) return fail(KVC_ERR_UNSUPPORTED, "max_q must be in [1, 65536]");
+    if (beacon_q && out_max_q < num_beacons) return fail(KVC_ERR_INVALID_ARGUMENT, "out_max_q is below num_beacons");
+    return cuda_status(kvc::launch_beacon(q, num_q, num_seqs, num_layers, num_q_heads, head_dim, max_q,
+                                          dtype == KVC_BF16, beacons, counts, num_beacons, beacon_q, out_max_q,
+                                          d_status, (cudaStream_t)stream),
+                       "kvc_beacon_update launch");
+}
+
 kvc_status kvc_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params *params,
                             kvc_stream_t stream) {
     g_err[0] = 0;

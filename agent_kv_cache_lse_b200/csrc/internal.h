@@ -47,6 +47,10 @@ cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const in
                            const int32_t *num_moves, const int32_t *new_len, float *crf, int32_t *freed,
                            int64_t freed_capacity, int64_t *num_freed, int64_t *row_offsets,
                            int32_t *status, cudaStream_t stream);
+cudaError_t launch_beacon(const void *q, const int32_t *num_q, int32_t num_seqs, int32_t num_layers,
+                          int32_t num_q_heads, int32_t head_dim, int32_t max_q, bool bf16, float *beacons,
+                          int32_t *counts, int32_t num_beacons, void *beacon_q, int32_t out_max_q, int32_t *status,
+                          cudaStream_t stream);
 cudaError_t launch_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params &p,
                                 cudaStream_t stream);
 cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab, void *state,

@@ -28,7 +28,7 @@ DEV_CODES = {0: "ok", 1: "bad page", 2: "bad length", 3: "non-finite value", 4: 
 EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse", "kvc_score_from_lse",
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
-           "kvc_confidence_ratchet"]
+           "kvc_confidence_ratchet", "kvc_beacon_update"]
 
 
 class KvcCache(ctypes.Structure):
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
             "kvc_ratchet_state_bytes": (ctypes.c_size_t, [i32, pr]),
             "kvc_ratchet_init": (ctypes.c_int, [vp, vp, i32, pr, vp]),
             "kvc_confidence_ratchet": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, pr, vp, vp]),
+            "kvc_beacon_update": (ctypes.c_int, [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp, vp, i32, vp, i32,
+                                                 vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -247,6 +249,19 @@ def kvc_confidence_ratchet(logits: torch.Tensor, state: torch.Tensor, budget: to
     _check(lib().kvc_confidence_ratchet(_ptr(logits), S, T, V, _ptr(state), _ptr(budget), _ptr(confidence_out),
                                         ctypes.byref(params), _ptr(d_status), _stream(stream)),
            "kvc_confidence_ratchet")
+
+
+def kvc_beacon_update(q: torch.Tensor, num_q: torch.Tensor, beacons: torch.Tensor, counts: torch.Tensor,
+                      beacon_q: Optional[torch.Tensor] = None, d_status=None, stream=None):
+    """q: [S][L][max_q][Hq][D] (bf16 or fp32); beacons: [S][L][Hq][B][D] fp32; counts: [S][L][Hq][B] int32;
+    beacon_q: optional [S][L][out_max_q][Hq][D] in q's dtype (rows 0..B-1 receive the beacons)."""
+    S, L, max_q, Hq, D = q.shape
+    B = beacons.shape[3]
+    dt = 1 if q.dtype == torch.bfloat16 else 0
+    out_max_q = beacon_q.shape[2] if beacon_q is not None else 0
+    _check(lib().kvc_beacon_update(_ptr(q), _ptr(num_q), S, L, Hq, D, max_q, dt, _ptr(beacons), _ptr(counts), B,
+                                   _ptr(beacon_q), out_max_q, _ptr(d_status), _stream(stream)),
+           "kvc_beacon_update")
 
 
 def ratchet_seq_states(state: torch.Tensor, num_seqs: int):

@@ -469,6 +469,49 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_beacon(args, device):
+    """Beacon-query maintenance on the streaming shape (8 sequences, 1 layer, 28 query heads, head_dim 128,
+    16 beacons per group, 64 new queries per group per round): rounds per second of kvc_beacon_update, with
+    the L2 cache flushed before every timed call; a separate line, not the eviction round."""
+    from agent_kv_cache_lse_b200 import kvc
+    S, L, Hq, D, B, m = 8, 1, 28, 128, 16, 64
+    gen = torch.Generator(device=device).manual_seed(4)
+    q = torch.randn((S, L, m, Hq, D), generator=gen, device=device).to(torch.bfloat16)
+    num_q = torch.full((S,), m, dtype=torch.int32, device=device)
+    beacons = torch.zeros((S, L, Hq, B, D), device=device)
+    counts = torch.zeros((S, L, Hq, B), dtype=torch.int32, device=device)
+    out = torch.zeros((S, L, B + 32, Hq, D), dtype=torch.bfloat16, device=device)
+    st = torch.zeros(2, dtype=torch.int32, device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    for _ in range(max(3, args.warmup)):
+        kvc.kvc_beacon_update(q, num_q, beacons, counts, out, st)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvc.kvc_beacon_update(q, num_q, beacons, counts, out, st)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    assert int(st[0]) == 0
+    ms = float(np.median(ts))
+    groups = S * L * Hq
+    algo = (S * L * m * Hq * D * 2) + groups * B * D * 4 * 2 + groups * B * 4 * 2 + S * L * B * Hq * D * 2
+    hbm, _, _, kind = peaks()
+    achieved = algo / (ms / 1e3) / 1e9
+    return {"metric": "beacon queries folded per second (streaming shape)", "value": groups * m / (ms / 1e3),
+            "unit": "queries/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16 queries, fp32 beacons", "data": "synthetic",
+            "config": {"workload": "beacon maintenance: 8 seqs x 1 layer x 28 q heads, head_dim 128, 16 beacons, "
+                                   "64 new queries per group", "l2": "flushed (256 MB write) before every call"},
+            "roofline": {"kernel": "beacon_kernel (kvc_beacon_update)", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak_source": f"{kind} HBM copy", "bytes_per_launch": algo},
+            "gpu_launches": args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -477,6 +520,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
+    ap.add_argument("--beacon", action="store_true", help="time beacon-query maintenance instead of the round")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -492,7 +536,7 @@ def main():
     device = torch.device("cuda", torch.cuda.current_device())
     from agent_kv_cache_lse_b200 import kvc
     kvc.lib()   # raises if the CUDA library is missing
-    line = run_ours(args, rank, world, device)
+    line = run_beacon(args, device) if args.beacon else run_ours(args, rank, world, device)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

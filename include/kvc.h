@@ -23,6 +23,10 @@
  *   5. kvc_compact_pages       one parallel in-place copy pass; shrunk block table
  *                              and freed-page list ("ActKV Dissected", Component 3)
  *
+ * Next to the path, building its query set:
+ *      kvc_beacon_update       beacon queries kept by online k-means over each
+ *                              group's past queries ("BeaconKV", Key ideas)
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Every pointer inside the structures and every array argument is DEVICE memory
@@ -286,6 +290,41 @@ kvc_status kvc_confidence_ratchet(const float *logits, int32_t num_seqs, int32_t
                                   void *state, int32_t *budget, float *confidence_out,
                                   const kvc_ratchet_params *params, int32_t *d_status,
                                   kvc_stream_t stream);
+
+/*
+ * Beacon queries ("BeaconKV Compresses KV Cache for Long-Reasoning Models with Beacon
+ * Queries", Key ideas: revisit-related queries form a few similarity groups, a representative
+ * of each group stands in for the query history, and these beacon queries join the recent
+ * queries in the query set).  The page does not say how the groups are found; here each
+ * group (sequence, layer, query head) keeps num_beacons beacons by online (mini-batch)
+ * k-means, and every call folds in that group's new queries:
+ *   1. beacons with count 0 are seeded, in index order, with the first new queries
+ *      (the j-th empty beacon takes query j);
+ *   2. every new query joins its nearest beacon among those with a count or a seed:
+ *      squared Euclidean distance summed over d = 0..head_dim-1 in order, with the
+ *      difference, the square and each partial sum rounded to fp32 separately (no fused
+ *      multiply-add); the lower beacon index wins a tie;
+ *   3. every beacon that drew new queries becomes the fp32 mean of all it has absorbed,
+ *      in a fixed order: S = c * n, S += each of its new queries in query order,
+ *      c = S / (n + drawn), n += drawn.  A beacon that drew nothing keeps its value (a seed
+ *      that drew nothing keeps count 0 and is seeded afresh next call).
+ * q:          new queries in the query-set layout [num_seqs][num_layers][max_q][num_q_heads]
+ *             [head_dim], `dtype` KVC_BF16 or KVC_F32; sequence s brings num_q[s] of them
+ *             (values above max_q are clamped, negative ones count as 0).
+ * beacons:    [num_seqs][num_layers][num_q_heads][num_beacons][head_dim] fp32, in/out.
+ * counts:     [num_seqs][num_layers][num_q_heads][num_beacons] int32, in/out; zero both
+ *             arrays to start a group empty.
+ * beacon_q:   NULL, or an output query set [num_seqs][num_layers][out_max_q][num_q_heads]
+ *             [head_dim] in `dtype` whose rows 0..num_beacons-1 receive the beacons (rounded
+ *             to nearest even for bf16), ready to lead the next round's query set; the
+ *             other rows are not touched.
+ * Limits: num_beacons in [1, 64], head_dim in [1, 256], max_q in [1, 65536], out_max_q >=
+ * num_beacons; otherwise KVC_ERR_INVALID_ARGUMENT or KVC_ERR_UNSUPPORTED.  One CTA per group.
+ */
+kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_seqs, int32_t num_layers,
+                             int32_t num_q_heads, int32_t head_dim, int32_t max_q, kvc_dtype dtype,
+                             float *beacons, int32_t *counts, int32_t num_beacons, void *beacon_q,
+                             int32_t out_max_q, int32_t *d_status, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -120,3 +120,18 @@ def test_bench_traffic_follows_kernel_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic() is None
     prof.write_text(f"source: {src}\nsource_sha256: {hashlib.sha256(b'x').hexdigest()}\ndram_bytes_per_launch: 5\n")
     assert bench.profiled_traffic() == 5
+
+
+def test_beacon_update_host_validation():
+    """Bad sizes are refused before anything reaches the device (fake pointers are never dereferenced)."""
+    from agent_kv_cache_lse_b200 import kvc
+    L = kvc.lib()
+    fake = ctypes.c_void_p(256)
+    call = lambda **kw: L.kvc_beacon_update(kw.get("q", fake), fake, kw.get("S", 1), 1, 1, kw.get("D", 128),
+                                            kw.get("mq", 8), kw.get("dt", 1), fake, fake, kw.get("B", 4),
+                                            kw.get("out", None), kw.get("omq", 0), None, None)
+    assert call(q=None) == 1                       # KVC_ERR_INVALID_ARGUMENT
+    assert call(B=0) == 2 and call(B=65) == 2      # KVC_ERR_UNSUPPORTED
+    assert call(D=300) == 2 and call(mq=70000) == 2 and call(dt=7) == 2
+    assert call(S=0) == 1
+    assert call(out=fake, omq=2) == 1              # output rows fewer than beacons
