@@ -193,6 +193,25 @@ kvc_status kvc_select_budget(const kvc_cache *cache, const float *crf, const int
                        "kvc_select_budget launch");
 }
 
+kvc_status kvc_lrfu_select(const kvc_cache *cache, const float *scores, float *crf, float lambda, float hit_mass,
+                           int32_t dt_rounds, uint32_t flags, const int32_t *budget, uint32_t protect_label_mask,
+                           uint8_t *keep, int32_t *kept, int32_t *d_status, kvc_stream_t stream) {
+    g_err[0] = 0;
+    kvc::CacheView c;
+    kvc_status s = view_cache(cache, c, false);
+    if (s != KVC_OK) return s;
+    if (!scores || !crf) return fail(KVC_ERR_INVALID_ARGUMENT, "scores and crf are required");
+    if (!budget || !keep || !kept) return fail(KVC_ERR_INVALID_ARGUMENT, "budget, keep and kept are required");
+    if (!(lambda >= 0.f) || !std::isfinite(lambda)) return fail(KVC_ERR_INVALID_ARGUMENT, "lambda must be >= 0");
+    if (!(hit_mass > 0.f) || !std::isfinite(hit_mass)) return fail(KVC_ERR_INVALID_ARGUMENT, "hit_mass must be > 0");
+    if (dt_rounds < 0) return fail(KVC_ERR_INVALID_ARGUMENT, "dt_rounds must be >= 0");
+    if (flags & ~KVC_HIT_BINARY) return fail(KVC_ERR_INVALID_ARGUMENT, "unknown flags");
+    const float decay = (float)std::exp2(-(double)lambda * (double)dt_rounds);
+    return cuda_status(kvc::launch_lrfu_select(c, scores, crf, decay, hit_mass, (flags & KVC_HIT_BINARY) != 0, budget,
+                                               protect_label_mask, keep, kept, d_status, (cudaStream_t)stream),
+                       "kvc_lrfu_select launch");
+}
+
 kvc_status kvc_plan_slots(const kvc_cache *cache, const uint8_t *keep, const int32_t *kept, int32_t *move_src,
                           int32_t *move_dst, int32_t *num_moves, int32_t *d_status, kvc_stream_t stream) {
     g_err[0] = 0;

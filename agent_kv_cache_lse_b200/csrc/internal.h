@@ -41,6 +41,9 @@ cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, flo
                         bool binary, int32_t *status, cudaStream_t stream);
 cudaError_t launch_select(const CacheView &c, const float *crf, const int32_t *budget, uint32_t protect,
                           uint8_t *keep, int32_t *kept, int32_t *status, cudaStream_t stream);
+cudaError_t launch_lrfu_select(const CacheView &c, const float *scores, float *crf, float decay, float hit_mass,
+                               bool binary, const int32_t *budget, uint32_t protect, uint8_t *keep, int32_t *kept,
+                               int32_t *status, cudaStream_t stream);
 cudaError_t launch_plan(const CacheView &c, const uint8_t *keep, const int32_t *kept, int32_t *move_src,
                         int32_t *move_dst, int32_t *num_moves, int32_t *status, cudaStream_t stream);
 cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const int32_t *move_dst,

@@ -10,157 +10,16 @@
 // 64-bit fixed-point integers (scores scaled by a power of two so the row maximum is
 // just under 2^48): integer sums make the search independent of summation order, so
 // the result is the same run to run.
-#include "internal.h"
-#include "rowcluster.cuh"
+
+#include "rowsteps.cuh"
 
 namespace kvc {
 namespace {
 
-constexpr int kThreads = 512;
-
-struct LrfuArgs {
-    CacheView c;
-    const float *scores;
-    float *crf;
-    float decay;      // 2^(-lambda * dt)
-    float hit_mass;
-    int binary;
-    int32_t *status;
-    int slice_cap;    // scores cached in shared memory when a CTA's slice fits
-    int weight_cap;   // fixed-point masses cached too when the slice fits this
-};
-
-__global__ void __launch_bounds__(kThreads, 1) lrfu_kernel(LrfuArgs a) {
+__global__ void __launch_bounds__(kRowThreads, 1) lrfu_kernel(LrfuArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    RowShared &sh = *reinterpret_cast<RowShared *>(smem_raw);
-    uint32_t *kc = reinterpret_cast<uint32_t *>(smem_raw + sizeof(RowShared));
-    unsigned long long *qw = reinterpret_cast<unsigned long long *>(
-        smem_raw + sizeof(RowShared) + (((size_t)a.slice_cap * 4 + 15) & ~(size_t)15));
     RowCtx rc = row_ctx();
-    const int row = blockIdx.x / rc.nranks;
-    const CacheView &c = a.c;
-    const int n = c.row_len[row];
-    if (n < 0 || n > c.max_slots) {
-        if (rc.rank == 0 && threadIdx.x == 0) report(a.status, KVC_DEV_BAD_LENGTH, row);
-        return;  // uniform across the cluster: no collective has started
-    }
-    const int per = (n + rc.nranks - 1) / rc.nranks;
-    const int lo = min(n, rc.rank * per), hi = min(n, lo + per);
-    const float *s = a.scores + (int64_t)row * c.max_slots;
-    float *crf = a.crf + (int64_t)row * c.max_slots;
-    const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots;
-    const bool cached = per <= a.slice_cap;
-    const bool wcached = cached && per <= a.weight_cap;
-
-    // stage the slice (raw fp32 bits, sign cleared so -0.0 ranks as 0), validate, row maximum
-    int bad = 0;
-    float mx = 0.f;
-    for (int base = lo + threadIdx.x; base < hi; base += 8 * blockDim.x) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {  // eight independent loads in flight before any is used
-            const int i = base + u * blockDim.x;
-            v[u] = i < hi ? s[i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = base + u * blockDim.x;
-            if (i < hi) {
-                if (!is_finite(v[u]) || v[u] < 0.f) bad = 1;
-                mx = fmaxf(mx, v[u]);
-                if (cached) kc[i - lo] = __float_as_uint(v[u]) & 0x7fffffffu;
-            }
-        }
-    }
-    row_max_or(rc, sh, mx, bad);
-    if (bad) {
-        if (rc.rank == 0 && threadIdx.x == 0) report(a.status, KVC_DEV_NONFINITE, row);
-        rc.cl.sync();
-        return;
-    }
-    auto skey = [&](int i) -> uint32_t { return cached ? kc[i - lo] : (__float_as_uint(s[i]) & 0x7fffffffu); };
-    auto sval = [&](int i) -> float { return __uint_as_float(skey(i)); };
-
-    uint32_t T = 0xffffffffu;  // threshold key; 0xffffffff: no hits
-    uint32_t PK = 0;
-    int tie_mode = 0;          // 0: every key == T is a hit; 1: decided by position; 2: then by slot order
-    unsigned long long slot_need = 0;
-    if (a.hit_mass >= 1.f) {
-        T = 1u;                // every positive score is a hit
-    } else if (mx > 0.f) {
-        int E;
-        frexpf(mx, &E);
-        const int e = 48 - E;
-        auto q = [&](int i) -> unsigned long long { return (unsigned long long)ldexp((double)sval(i), e); };
-        unsigned long long part = 0;
-        for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-            const unsigned long long w = q(i);
-            part += w;
-            if (wcached) qw[i - lo] = w;  // each pass of the search below reads it instead of recomputing
-        }
-        const unsigned long long Sq = row_sum_u64(rc, sh, part);  // its cluster barrier also orders qw
-        auto qv = [&](int i) -> unsigned long long { return wcached ? qw[i - lo] : q(i); };
-        unsigned long long target = (unsigned long long)ceil((double)a.hit_mass * (double)Sq);
-        if (target > Sq) target = Sq;
-        if (target >= 1) {
-            const RadixResult r = row_radix_desc<true>(rc, sh, lo, hi, target, skey, qv,
-                                                       [&](int i) { return skey(i) != 0u; });
-            T = r.key;
-            const unsigned long long qT = (unsigned long long)ldexp((double)__uint_as_float(T), e);
-            const unsigned long long rem = target - r.above;
-            unsigned long long need = qT > 0 ? (rem + qT - 1) / qT : r.eq_count;
-            if (need > r.eq_count) need = r.eq_count;
-            if (need < r.eq_count) {
-                const RadixResult r2 = row_radix_desc<false>(
-                    rc, sh, lo, hi, need, [&](int i) { return pos_desc_key(pos[i]); }, [](int) { return 1ull; },
-                    [&](int i) { return skey(i) == T; });
-                PK = r2.key;
-                tie_mode = 1;
-                const unsigned long long need2 = need - r2.above;
-                if (need2 < r2.eq_count) {
-                    tie_mode = 2;
-                    slot_need = need2;
-                }
-            }
-        }
-    }
-    auto is_hit = [&](int i) -> int {
-        const uint32_t k = skey(i);
-        if (k == 0u) return 0;
-        if (k > T) return 1;
-        if (k < T) return 0;
-        if (tie_mode == 0) return 1;
-        const uint32_t pk = pos_desc_key(pos[i]);
-        if (pk > PK) return 1;
-        if (pk < PK) return 0;
-        return tie_mode == 1 ? 1 : -1;
-    };
-    auto update = [&](int i, int hit) {
-        const float h = hit ? (a.binary ? 1.f : sval(i)) : 0.f;
-        crf[i] = fmaf(a.decay, crf[i], h);
-    };
-    if (tie_mode == 2) {
-        // entries equal in score and position: the first ones in slot order, across the cluster
-        row_ordered_ranks(rc, sh, lo, hi, [&](int i) { return is_hit(i) < 0; },
-                          [&](int i, int rank) { update(i, (unsigned long long)rank < slot_need); });
-    }
-    for (int base = lo + threadIdx.x; base < hi; base += 8 * blockDim.x) {
-        float old[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = base + u * blockDim.x;
-            old[u] = i < hi ? crf[i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = base + u * blockDim.x;
-            if (i < hi) {
-                const int hit = is_hit(i);
-                if (hit >= 0) crf[i] = fmaf(a.decay, old[u], hit ? (a.binary ? 1.f : sval(i)) : 0.f);
-            }
-        }
-    }
-    rc.cl.sync();  // peers may still read this CTA's shared memory
+    lrfu_row(a, rc, smem_raw);
 }
 
 }  // namespace
@@ -182,7 +41,7 @@ cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, flo
     LrfuArgs a{c, scores, crf, decay, hit_mass, binary ? 1 : 0, status, cap, wcap};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(c.rows * C));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kRowThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

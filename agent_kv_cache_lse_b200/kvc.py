@@ -28,7 +28,7 @@ DEV_CODES = {0: "ok", 1: "bad page", 2: "bad length", 3: "non-finite value", 4: 
 EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse", "kvc_score_from_lse",
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
-           "kvc_confidence_ratchet", "kvc_beacon_update"]
+           "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select"]
 
 
 class KvcCache(ctypes.Structure):
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
             "kvc_score_from_lse": (ctypes.c_int, [pc, pq, vp, u32, vp, vp]),
             "kvc_lrfu_update": (ctypes.c_int, [pc, vp, vp, f32, f32, i32, u32, vp, vp]),
             "kvc_select_budget": (ctypes.c_int, [pc, vp, vp, u32, vp, vp, vp, vp]),
+            "kvc_lrfu_select": (ctypes.c_int, [pc, vp, vp, f32, f32, i32, u32, vp, u32, vp, vp, vp, vp]),
             "kvc_plan_slots": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, vp]),
             "kvc_compact_workspace_bytes": (ctypes.c_size_t, [i32]),
             "kvc_compact_pages": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, i64, vp, vp, ctypes.c_size_t, vp, vp]),
@@ -194,6 +195,17 @@ def kvc_select_budget(cache: Cache, crf: torch.Tensor, budget: torch.Tensor, kee
     cs = cache.struct()
     _check(lib().kvc_select_budget(ctypes.byref(cs), _ptr(crf), _ptr(budget), protect_label_mask, _ptr(keep),
                                    _ptr(kept), _ptr(d_status), _stream(stream)), "kvc_select_budget")
+
+
+def kvc_lrfu_select(cache: Cache, scores: torch.Tensor, crf: torch.Tensor, budget: torch.Tensor, keep: torch.Tensor,
+                    kept: torch.Tensor, lam: float = 0.5, hit_mass: float = 0.9, dt_rounds: int = 1, flags: int = 0,
+                    protect_label_mask: int = 0, d_status=None, stream=None):
+    """kvc_lrfu_update followed by kvc_select_budget, in one launch."""
+    cs = cache.struct()
+    _check(lib().kvc_lrfu_select(ctypes.byref(cs), _ptr(scores), _ptr(crf), lam, hit_mass, dt_rounds, flags,
+                                 _ptr(budget), protect_label_mask, _ptr(keep), _ptr(kept), _ptr(d_status),
+                                 _stream(stream)),
+           "kvc_lrfu_select")
 
 
 def kvc_plan_slots(cache: Cache, keep: torch.Tensor, kept: torch.Tensor, move_src: torch.Tensor,

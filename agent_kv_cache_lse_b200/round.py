@@ -3,8 +3,8 @@
 ``EvictionRound`` owns the per-round device buffers (scores, LRFU values, keep mask,
 slot plan, freed-page list, workspace, ratchet state) and enqueues, on one stream:
 
-  kvc_confidence_ratchet -> kvc_score_from_lse -> kvc_lrfu_update -> kvc_select_budget
-  -> kvc_plan_slots -> kvc_compact_pages
+  kvc_confidence_ratchet -> kvc_score_from_lse -> kvc_lrfu_select (LRFU update and
+  top-budget selection in one launch) -> kvc_plan_slots -> kvc_compact_pages
 
 ("ActKV Dissected": Component 2 budget, Component 1 scoring and LRFU, Component 3
 slot plan and in-place compaction).  Nothing here computes; it only allocates with
@@ -21,7 +21,7 @@ from . import kvc
 
 
 class EvictionRound:
-    KERNELS_PER_ROUND = 8  # ratchet 2, score 1, lrfu 1, select 1, plan 1, compact 2
+    KERNELS_PER_ROUND = 7  # ratchet 2, score 1, lrfu + select 1, plan 1, compact 2
 
     def __init__(self, cache: kvc.Cache, params: Optional[kvc.KvcRatchetParams] = None,
                  freed_capacity: Optional[int] = None, device="cuda"):
@@ -60,8 +60,8 @@ class EvictionRound:
             kvc.kvc_confidence_ratchet(logits, self.state, self.budget, self.params, confidence_out, self.status,
                                        stream)
         kvc.kvc_score_from_lse(c, queries, self.scores, score_flags, self.status, stream)
-        kvc.kvc_lrfu_update(c, self.scores, self.crf, lam, hit_mass, 1, 0, self.status, stream)
-        kvc.kvc_select_budget(c, self.crf, self.budget, self.keep, self.kept, protect_label_mask, self.status, stream)
+        kvc.kvc_lrfu_select(c, self.scores, self.crf, self.budget, self.keep, self.kept, lam, hit_mass, 1, 0,
+                            protect_label_mask, self.status, stream)
         kvc.kvc_plan_slots(c, self.keep, self.kept, self.move_src, self.move_dst, self.num_moves, self.status, stream)
         kvc.kvc_compact_pages(c, self.move_src, self.move_dst, self.num_moves, self.kept, self.crf, self.freed,
                               self.num_freed, self.workspace, self.status, stream)

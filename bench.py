@@ -198,8 +198,7 @@ def run_ours(args, rank, world, device):
         kvc.kvc_score_from_lse(cache, queries, rnd.scores, 0, rnd.status)
         if e is not None:
             e[2].record()
-        kvc.kvc_lrfu_update(cache, rnd.scores, rnd.crf, 0.5, 0.9, 1, 0, rnd.status)
-        kvc.kvc_select_budget(cache, rnd.crf, rnd.budget, rnd.keep, rnd.kept, 0, rnd.status)
+        kvc.kvc_lrfu_select(cache, rnd.scores, rnd.crf, rnd.budget, rnd.keep, rnd.kept, 0.5, 0.9, 1, 0, 0, rnd.status)
         kvc.kvc_plan_slots(cache, rnd.keep, rnd.kept, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.status)
         kvc.kvc_compact_pages(cache, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.kept, rnd.crf, rnd.freed,
                               rnd.num_freed, rnd.workspace, rnd.status)
@@ -214,7 +213,7 @@ def run_ours(args, rank, world, device):
     if code != 0:
         raise RuntimeError(f"device status {rnd.device_status()} during warm-up")
 
-    # the round as one CUDA graph (the six calls, eight kernels), with timing events captured as nodes
+    # the round as one CUDA graph (five calls, seven kernels), with timing events captured as nodes
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     graph = None
     if not args.no_graph:
@@ -304,7 +303,7 @@ def run_ours(args, rank, world, device):
     return line
 
 
-EvictionRound_KERNELS = 8
+EvictionRound_KERNELS = 7
 
 SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
 
@@ -519,7 +518,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
-    ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
+    ap.add_argument("--no-graph", action="store_true", help="launch the five calls directly instead of a CUDA graph")
     ap.add_argument("--beacon", action="store_true", help="time beacon-query maintenance instead of the round")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

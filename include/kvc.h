@@ -220,6 +220,18 @@ kvc_status kvc_select_budget(const kvc_cache *cache, const float *crf, const int
                              int32_t *d_status, kvc_stream_t stream);
 
 /*
+ * Steps 2 and 3b in one launch: the same arguments, the same checks and the same results as
+ * kvc_lrfu_update(cache, scores, crf, lambda, hit_mass, dt_rounds, flags, ...) followed by
+ * kvc_select_budget(cache, crf, budget, protect_label_mask, keep, kept, ...) on one stream.
+ * One cluster per row runs both: the selection reads the LRFU values the cluster has just
+ * written, with no second launch.  (A system-level fusion of two steps of "ActKV Dissected",
+ * Component 1 and Summary; the pages have no counterpart of the entry point itself.)
+ */
+kvc_status kvc_lrfu_select(const kvc_cache *cache, const float *scores, float *crf, float lambda, float hit_mass,
+                           int32_t dt_rounds, uint32_t flags, const int32_t *budget, uint32_t protect_label_mask,
+                           uint8_t *keep, int32_t *kept, int32_t *d_status, kvc_stream_t stream);
+
+/*
  * Step 4: with m = kept[row], the holes are the slots i < m with keep 0 and the
  * survivors are the slots i >= m with keep 1, both ascending; move j copies survivor j
  * into hole j.  move_src/move_dst: [rows][max_slots] int32 (first num_moves[row] valid).

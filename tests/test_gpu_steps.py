@@ -219,6 +219,43 @@ def test_lrfu_parity(mode, variant):
 
 # ----------------------------------------------------------------------------- plan + compaction
 
+@pytest.mark.parametrize("mode", ["lognormal", "ties", "sparse", "equal"])
+def test_lrfu_select_fused_matches_separate(mode):
+    """kvc_lrfu_select equals kvc_lrfu_update then kvc_select_budget: LRFU values bit for bit, the same keep
+    mask and counts, with protected labels; and the selection it makes equals the oracle's on those values."""
+    rng = np.random.default_rng(41)
+    lengths = [0, 1, 16, 257, 5000, 33000]
+    ms = 33008
+    c = bare_cache(lengths, ms, S=len(lengths))
+    s = np.zeros((len(lengths), ms), dtype=np.float32)
+    crf0 = np.zeros((len(lengths), ms), dtype=np.float32)
+    for r, n in enumerate(lengths):
+        s[r, :n] = _row_values(rng, n, mode)
+        crf0[r, :n] = _row_values(rng, n, mode)
+    budgets = torch.tensor([3, 0, 5, 100, 512, 2048], dtype=torch.int32, device=DEV)
+    sd = torch.from_numpy(s).to(DEV)
+    outs = []
+    for fused in (False, True):
+        crf = torch.from_numpy(crf0.copy()).to(DEV)
+        keep = torch.full((len(lengths), ms), 9, dtype=torch.uint8, device=DEV)
+        kept = torch.zeros(len(lengths), dtype=torch.int32, device=DEV)
+        st = torch.zeros(2, dtype=torch.int32, device=DEV)
+        if fused:
+            kvc.kvc_lrfu_select(c, sd, crf, budgets, keep, kept, 0.5, HIT, 1, 0, 1 << 2, st)
+        else:
+            kvc.kvc_lrfu_update(c, sd, crf, 0.5, HIT, 1, 0, st)
+            kvc.kvc_select_budget(c, crf, budgets, keep, kept, 1 << 2, st)
+        torch.cuda.synchronize()
+        outs.append((crf.cpu().numpy(), keep.cpu().numpy(), kept.cpu().numpy(), st.cpu().tolist()))
+    (c0, k0, n0, s0), (c1, k1, n1, s1) = outs
+    assert np.array_equal(c0.view(np.uint32), c1.view(np.uint32))
+    assert np.array_equal(k0, k1) and np.array_equal(n0, n1) and s0 == s1 == [0, 0]
+    pos, lab = c.slot_pos.cpu().numpy(), c.slot_label.cpu().numpy()
+    for r, n in enumerate(lengths):
+        ok = opath.select_budget(c1[r, :n].astype(np.float64), pos[r, :n], int(budgets[r]), lab[r, :n], 1 << 2)
+        assert np.array_equal(k1[r, :n].astype(bool), ok), f"row {r}"
+
+
 def _masks(rng, lengths, mode):
     keeps = []
     for n in lengths:
