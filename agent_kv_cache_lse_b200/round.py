@@ -1,10 +1,13 @@
-"""One eviction round over a paged cache: the six C-ABI calls in path order.
+"""One eviction round over a paged cache: the C-ABI calls in path order.
 
 ``EvictionRound`` owns the per-round device buffers (scores, LRFU values, keep mask,
-slot plan, freed-page list, workspace, ratchet state) and enqueues, on one stream:
+slot plan, freed-page list, workspace, ratchet state) and enqueues, on the caller's stream:
 
-  kvc_confidence_ratchet -> kvc_score_from_lse -> kvc_lrfu_select (LRFU update and
-  top-budget selection in one launch) -> kvc_plan_slots -> kvc_compact_pages
+  kvc_score_from_lse -> (kvc_confidence_ratchet on a second stream | kvc_lrfu_update)
+  -> kvc_select_budget -> kvc_plan_slots -> kvc_compact_pages
+
+and, in a round without logits (budget unchanged), kvc_lrfu_select (LRFU update and
+top-budget selection in one launch) in place of the middle three.
 
 ("ActKV Dissected": Component 2 budget, Component 1 scoring and LRFU, Component 3
 slot plan and in-place compaction).  Nothing here computes; it only allocates with
@@ -21,7 +24,7 @@ from . import kvc
 
 
 class EvictionRound:
-    KERNELS_PER_ROUND = 7  # ratchet 2, score 1, lrfu + select 1, plan 1, compact 2
+    KERNELS_PER_ROUND = 8  # ratchet 2, score 1, lrfu 1, select 1, plan 1, compact 2 (7 without logits)
 
     def __init__(self, cache: kvc.Cache, params: Optional[kvc.KvcRatchetParams] = None,
                  freed_capacity: Optional[int] = None, device="cuda"):
@@ -47,6 +50,8 @@ class EvictionRound:
         nb = kvc.kvc_ratchet_state_bytes(S, self.params)
         self.state = torch.zeros(((nb + 15) // 16) * 16, dtype=torch.uint8, device=dev)
         kvc.kvc_ratchet_init(self.state, self.budget, S, self.params)
+        self._side = torch.cuda.Stream(device=dev)
+        self._fork, self._join = torch.cuda.Event(), torch.cuda.Event()
 
     def reset_ratchet(self, stream=None):
         kvc.kvc_ratchet_init(self.state, self.budget, self.cache.num_seqs, self.params, stream)
@@ -54,17 +59,29 @@ class EvictionRound:
     def run(self, queries: kvc.QuerySet, logits: Optional[torch.Tensor] = None, lam: float = 0.5,
             hit_mass: float = 0.9, score_flags: int = 0, protect_label_mask: int = 0,
             confidence_out: Optional[torch.Tensor] = None, stream=None):
-        """Enqueue one round.  logits [S, steps, V] fp32 drive the ratchet (None: budget unchanged)."""
+        """Enqueue one round.  logits [S, steps, V] fp32 drive the ratchet (None: budget unchanged).
+
+        With logits, the ratchet runs on a second stream beside the LRFU update (neither needs the other;
+        the selection needs both), forked after the scores and joined before the selection."""
         c = self.cache
+        main = stream if stream is not None else torch.cuda.current_stream()
+        kvc.kvc_score_from_lse(c, queries, self.scores, score_flags, self.status, main)
         if logits is not None:
+            # the LRFU update goes first so that its clusters take their SMs before the ratchet's CTAs spread
+            self._fork.record(main)
+            kvc.kvc_lrfu_update(c, self.scores, self.crf, lam, hit_mass, 1, 0, self.status, main)
+            self._side.wait_event(self._fork)
             kvc.kvc_confidence_ratchet(logits, self.state, self.budget, self.params, confidence_out, self.status,
-                                       stream)
-        kvc.kvc_score_from_lse(c, queries, self.scores, score_flags, self.status, stream)
-        kvc.kvc_lrfu_select(c, self.scores, self.crf, self.budget, self.keep, self.kept, lam, hit_mass, 1, 0,
-                            protect_label_mask, self.status, stream)
-        kvc.kvc_plan_slots(c, self.keep, self.kept, self.move_src, self.move_dst, self.num_moves, self.status, stream)
+                                       self._side)
+            self._join.record(self._side)
+            main.wait_event(self._join)
+            kvc.kvc_select_budget(c, self.crf, self.budget, self.keep, self.kept, protect_label_mask, self.status, main)
+        else:
+            kvc.kvc_lrfu_select(c, self.scores, self.crf, self.budget, self.keep, self.kept, lam, hit_mass, 1, 0,
+                                protect_label_mask, self.status, main)
+        kvc.kvc_plan_slots(c, self.keep, self.kept, self.move_src, self.move_dst, self.num_moves, self.status, main)
         kvc.kvc_compact_pages(c, self.move_src, self.move_dst, self.num_moves, self.kept, self.crf, self.freed,
-                              self.num_freed, self.workspace, self.status, stream)
+                              self.num_freed, self.workspace, self.status, main)
 
     def device_status(self):
         return kvc.device_status(self.status)
