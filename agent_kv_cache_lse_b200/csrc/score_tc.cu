@@ -367,6 +367,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t *qp = a.q.q_pos + (int64_t)seq * a.q.max_q;
         for (int j = lane * 32; j < a.q.max_q; j += 32 * 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(qp + j));
     }
+    // The first tile's sequence: the q_pos range of each of its query blocks, computed by the whole CTA (one
+    // load per thread and query) so that the decoder starts with it instead of gathering it alone.
+    int seq0 = -1, nq0 = 0;
+    if ((int64_t)blockIdx.x < a.total_tiles) {
+        seq0 = (int)(((int64_t)blockIdx.x / (c.num_layers * c.num_kv_heads)) / a.tiles_per_row);
+        nq0 = min(a.q.num_q[seq0], a.q.max_q);
+        for (int b = threadIdx.x; b < (nq0 + a.nqb - 1) / a.nqb; b += kThreads) {
+            ctl.blk_qmin[0][b] = INT32_MAX;
+            ctl.blk_qmax[0][b] = INT32_MIN;
+        }
+    }
+    __syncthreads();
+    if (seq0 >= 0) {
+        const int32_t *qrow = a.q.q_pos + (int64_t)seq0 * a.q.max_q;
+        for (int j = threadIdx.x; j < nq0; j += kThreads) {
+            const int p = qrow[j];
+            atomicMin(&ctl.blk_qmin[0][j / a.nqb], p);
+            atomicMax(&ctl.blk_qmax[0][j / a.nqb], p);
+        }
+    }
     // zero the operand buffers once so rows no load ever fills hold finite values
     for (int i = threadIdx.x; i < (2 * PL::kABytes + PL::kStages * PL::kBBytes) / 16; i += kThreads)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
@@ -481,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t mk = 0, mph = 0, tk = 0, tph = 0;
         // q_pos ranges of a sequence's blocks live in one of two buffers: the tile being produced and the one
         // decoded ahead of it may belong to different sequences
-        int cur_seq = -1, nblk = 0, nq = 0, sbuf = 1;
+        int cur_seq = seq0, nq = nq0, nblk = seq0 >= 0 ? (nq0 + nqb - 1) / nqb : 0, sbuf = 0;
         bool ok = true;
         const int mp = c.max_pages_per_row;
         const int64_t ms = c.max_slots;
