@@ -276,6 +276,29 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
                        "kvc_beacon_update launch");
 }
 
+kvc_status kvc_decode_attention(const kvc_cache *cache, const void *q, const int32_t *q_pos, int32_t num_q_heads,
+                                float *out, float *lse, float *scores, uint32_t flags, int32_t *d_status,
+                                kvc_stream_t stream) {
+    g_err[0] = 0;
+    kvc::CacheView c;
+    kvc_status s = view_cache(cache, c, true);
+    if (s != KVC_OK) return s;
+    if (!q || !q_pos || !out || !lse) return fail(KVC_ERR_INVALID_ARGUMENT, "q, q_pos, out and lse are required");
+    if (num_q_heads <= 0 || num_q_heads % c.num_kv_heads != 0)
+        return fail(KVC_ERR_INVALID_ARGUMENT, "num_q_heads must be a positive multiple of num_kv_heads");
+    if (flags & ~KVC_SCORE_ACCUMULATE) return fail(KVC_ERR_INVALID_ARGUMENT, "unknown flags");
+    const int group = num_q_heads / c.num_kv_heads;
+    if (group > 8) return fail(KVC_ERR_UNSUPPORTED, "at most 8 query heads per KV head");
+    const int cluster = kvc::decode_cluster(c, group);
+    if (cluster == 0)
+        return fail(KVC_ERR_UNSUPPORTED, "a row of %lld slots with %d query heads per KV head exceeds the logits buffer",
+                    (long long)c.max_slots, group);
+    return cuda_status(kvc::launch_decode(c, q, q_pos, num_q_heads, out, lse, scores,
+                                          (flags & KVC_SCORE_ACCUMULATE) != 0, d_status, (cudaStream_t)stream,
+                                          cluster),
+                       "kvc_decode_attention launch");
+}
+
 kvc_status kvc_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params *params,
                             kvc_stream_t stream) {
     g_err[0] = 0;

@@ -54,6 +54,12 @@ cudaError_t launch_beacon(const void *q, const int32_t *num_q, int32_t num_seqs,
                           int32_t num_q_heads, int32_t head_dim, int32_t max_q, bool bf16, float *beacons,
                           int32_t *counts, int32_t num_beacons, void *beacon_q, int32_t out_max_q, int32_t *status,
                           cudaStream_t stream);
+// Cluster size the decode kernel uses for this cache and group size; 0 when a row's logits
+// do not fit the shared memory of a cluster of 8 CTAs.
+int decode_cluster(const CacheView &c, int32_t group);
+cudaError_t launch_decode(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
+                          float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream,
+                          int cluster);
 cudaError_t launch_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params &p,
                                 cudaStream_t stream);
 cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab, void *state,

@@ -28,7 +28,7 @@ DEV_CODES = {0: "ok", 1: "bad page", 2: "bad length", 3: "non-finite value", 4: 
 EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse", "kvc_score_from_lse",
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
-           "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select"]
+           "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select", "kvc_decode_attention"]
 
 
 class KvcCache(ctypes.Structure):
@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
             "kvc_confidence_ratchet": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, pr, vp, vp]),
             "kvc_beacon_update": (ctypes.c_int, [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp, vp, i32, vp, i32,
                                                  vp, vp]),
+            "kvc_decode_attention": (ctypes.c_int, [pc, vp, vp, i32, vp, vp, vp, u32, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -274,6 +275,17 @@ def kvc_beacon_update(q: torch.Tensor, num_q: torch.Tensor, beacons: torch.Tenso
     _check(lib().kvc_beacon_update(_ptr(q), _ptr(num_q), S, L, Hq, D, max_q, dt, _ptr(beacons), _ptr(counts), B,
                                    _ptr(beacon_q), out_max_q, _ptr(d_status), _stream(stream)),
            "kvc_beacon_update")
+
+
+def kvc_decode_attention(cache: Cache, q: torch.Tensor, q_pos: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                         scores: Optional[torch.Tensor] = None, flags: int = 0, d_status=None, stream=None):
+    """One decode step with the scores folded in.  q: [S][L][Hq][D] in the cache dtype; q_pos: [S] int32;
+    out: [S][L][Hq][D] fp32; lse: [S][L][Hq] fp32; scores: optional [rows][max_slots] fp32
+    (KVC_SCORE_ACCUMULATE adds into it)."""
+    cs = cache.struct()
+    _check(lib().kvc_decode_attention(ctypes.byref(cs), _ptr(q), _ptr(q_pos), q.shape[2], _ptr(out), _ptr(lse),
+                                      _ptr(scores), flags, _ptr(d_status), _stream(stream)),
+           "kvc_decode_attention")
 
 
 def ratchet_seq_states(state: torch.Tensor, num_seqs: int):

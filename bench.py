@@ -524,6 +524,79 @@ def run_beacon(args, device):
             "gpu_launches": args.steps}
 
 
+def decode_workload(spec, device):
+    """Cache of a decode workload and the step's query (the first query of each sequence's set) at the next
+    position, so that every cached key is visible."""
+    from agent_kv_cache_lse_b200 import kvc, synth
+    layout = synth.make_layout(spec)
+    kp = synth.fill_pool(spec, layout, "k", device)
+    vp = synth.fill_pool(spec, layout, "v", device)
+    qs = synth.make_queries(spec, device)
+    cache = kvc.Cache(kp, vp, layout.block_table.to(device), layout.row_len.to(device), layout.slot_pos.to(device),
+                      layout.slot_label.to(device), spec.num_seqs, spec.num_layers, spec.num_kv_heads)
+    q = qs.q[:, :, 0].contiguous()
+    q_pos = torch.tensor(list(spec.ctx), dtype=torch.int32, device=device)
+    return cache, q, q_pos, int(layout.row_len.sum())
+
+
+def time_decode(args, spec, device, flush):
+    from agent_kv_cache_lse_b200 import kvc
+    cache, q, q_pos, entries = decode_workload(spec, device)
+    S, L, Hq, D = q.shape
+    out = torch.empty((S, L, Hq, D), device=device)
+    lse = torch.empty((S, L, Hq), device=device)
+    scores = torch.zeros((spec.rows, spec.max_slots), device=device)
+    st = torch.zeros(2, dtype=torch.int32, device=device)
+    for _ in range(max(3, args.warmup)):
+        kvc.kvc_decode_attention(cache, q, q_pos, out, lse, scores, kvc.KVC_SCORE_ACCUMULATE, st)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvc.kvc_decode_attention(cache, q, q_pos, out, lse, scores, kvc.KVC_SCORE_ACCUMULATE, st)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    assert int(st[0]) == 0, kvc.device_status(st)
+    elem = 2 if spec.dtype == "bf16" else 4
+    # per visible entry: K and V rows, its slot position, and the score's read-modify-write; per query head:
+    # the query, the output row and the LSE; per row: its length and block-table row
+    algo = (entries * (2 * D * elem + 4 + 8) + S * L * Hq * (D * elem + D * 4 + 4)
+            + spec.rows * (4 + spec.max_pages_per_row * 4))
+    ms = float(np.median(ts))
+    del cache
+    return ms, entries, algo, ts
+
+
+def run_decode(args, device):
+    """One decode step of paged attention with the scores folded in (kvc_decode_attention, accumulating into the
+    round's scores): KV entries attended and scored per second for one layer of the batch of 16 sequences
+    (context 8K-33K, 32 q / 8 KV heads, head_dim 128, bf16), L2 flushed before every call; the single Llama-3-8B
+    layer at 32K is timed beside it.  A separate line, not the eviction round."""
+    from agent_kv_cache_lse_b200 import synth
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    hbm, _, _, kind = peaks()
+    ms, entries, algo, ts = time_decode(args, synth.batch16(num_layers=1), device, flush)
+    ms1, entries1, algo1, _ = time_decode(args, synth.llama8b_layer(), device, flush)
+    achieved = algo / (ms / 1e3) / 1e9
+    p10, p50, p90 = (float(x) for x in np.percentile(ts, [10, 50, 90]))
+    return {"metric": "KV entries attended+scored/sec (fused decode step)", "value": entries / (ms / 1e3),
+            "unit": "entries/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_step_p10_p50_p90": [p10, p50, p90], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 K/V/Q, fp32 accumulate", "data": "synthetic",
+            "config": {"workload": "decode step, one layer of the batch of 16 sequences (context 8K-33K, "
+                                   f"{entries} cached entries), 32 q / 8 KV heads, head_dim 128, bf16, 16-token pages",
+                       "l2": "flushed (256 MB write) before every call"},
+            "single_layer_32k": {"entries": entries1, "ms": ms1, "entries_per_s": entries1 / (ms1 / 1e3),
+                                 "achieved_gbs": algo1 / (ms1 / 1e3) / 1e9},
+            "roofline": {"kernel": "decode_kernel (kvc_decode_attention)", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak_source": f"{kind} HBM copy", "bytes_per_launch": algo},
+            "gpu_launches": args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -533,6 +606,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
     ap.add_argument("--beacon", action="store_true", help="time beacon-query maintenance instead of the round")
+    ap.add_argument("--decode", action="store_true", help="time the fused decode step instead of the round")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -548,7 +622,12 @@ def main():
     device = torch.device("cuda", torch.cuda.current_device())
     from agent_kv_cache_lse_b200 import kvc
     kvc.lib()   # raises if the CUDA library is missing
-    line = run_beacon(args, device) if args.beacon else run_ours(args, rank, world, device)
+    if args.beacon:
+        line = run_beacon(args, device)
+    elif args.decode:
+        line = run_decode(args, device)
+    else:
+        line = run_ours(args, rank, world, device)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -338,6 +338,37 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
                              float *beacons, int32_t *counts, int32_t num_beacons, void *beacon_q,
                              int32_t out_max_q, int32_t *d_status, kvc_stream_t stream);
 
+/*
+ * One decode step of paged attention with the step's score contribution folded in
+ * ("ActKV Dissected", Component 3: the LSE is a byproduct of paged attention, so the
+ * query's attention probabilities are its logits minus the LSE, with no gather of the
+ * attention matrix and no recompute).  For every row (sequence, layer, KV head) and each
+ * query head g of its GQA group, over the row's slots i < row_len with slot_pos <= q_pos:
+ *     l[g, i] = q_g . k_i / sqrt(head_dim)
+ *     lse[g]  = log sum_i exp(l[g, i])                  (-inf when no key is visible)
+ *     out[g]  = sum_i exp(l[g, i] - lse[g]) v_i          (zeros when no key is visible)
+ *     scores[row][i] (+)= sum_g exp(l[g, i] - lse[g])     (0 for a hidden slot)
+ * q:       [num_seqs][num_layers][num_q_heads][head_dim] in the cache's dtype, one query
+ *          per (sequence, layer, head); query head h belongs to KV head h / (num_q_heads /
+ *          num_kv_heads).
+ * q_pos:   [num_seqs] int32 position of the step's token (INT32_MAX sees every slot).
+ * out:     [num_seqs][num_layers][num_q_heads][head_dim] fp32, written.
+ * lse:     [num_seqs][num_layers][num_q_heads] fp32 natural log, written.
+ * scores:  NULL (attention only) or [rows][max_pages_per_row * page_size] fp32, written
+ *          (added to with KVC_SCORE_ACCUMULATE) for slots < row_len only.
+ * flags:   0 or KVC_SCORE_ACCUMULATE.
+ * Limits:  num_q_heads / num_kv_heads <= 8, and the row's logits must fit a cluster of 8
+ *          CTAs: ceil(max_slots / 8) * G' * 4 bytes plus G * head_dim * 36 bytes within
+ *          200 KiB, G' being the group size rounded up to a power of two (max_slots up to
+ *          about 90k for G = 4); otherwise KVC_ERR_UNSUPPORTED.  d_status reports a bad page
+ *          or a bad row length; the affected row's results are then undefined.
+ * Every sum runs in a fixed order: results repeat bit for bit.  One cluster of up to 8 CTAs
+ * per row, exchanging maxima, sums and partial outputs through distributed shared memory.
+ */
+kvc_status kvc_decode_attention(const kvc_cache *cache, const void *q, const int32_t *q_pos, int32_t num_q_heads,
+                                float *out, float *lse, float *scores, uint32_t flags, int32_t *d_status,
+                                kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
