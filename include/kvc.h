@@ -357,11 +357,13 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
  * scores:  NULL (attention only) or [rows][max_pages_per_row * page_size] fp32, written
  *          (added to with KVC_SCORE_ACCUMULATE) for slots < row_len only.
  * flags:   0 or KVC_SCORE_ACCUMULATE.
- * Limits:  num_q_heads / num_kv_heads <= 8, and the row's logits must fit a cluster of 8
- *          CTAs: ceil(max_slots / 8) * G' * 4 bytes plus G * head_dim * 36 bytes within
- *          200 KiB, G' being the group size rounded up to a power of two (max_slots up to
- *          about 90k for G = 4); otherwise KVC_ERR_UNSUPPORTED.  d_status reports a bad page
- *          or a bad row length; the affected row's results are then undefined.
+ * Limits:  num_q_heads / num_kv_heads <= 8, and a CTA of the row's cluster (at most 8 CTAs)
+ *          must hold its slice's logits and positions, (G' + 1) * 4 * ceil(max_slots / 8) bytes
+ *          (G' = the group size rounded up to a power of two), beside two K/V stages per warp of
+ *          a chunk (up to 16 slots of one page), within 220 KiB: for bf16 and head_dim
+ *          128, max_slots up to about 37,000 at G = 4 and 94,000 at G = 1; otherwise
+ *          KVC_ERR_UNSUPPORTED.  d_status reports a bad page or a bad row length; the affected
+ *          row's results are then undefined.
  * Every sum runs in a fixed order: results repeat bit for bit.  One cluster of up to 8 CTAs
  * per row, exchanging maxima, sums and partial outputs through distributed shared memory.
  */

@@ -190,6 +190,17 @@ def test_decode_host_validation():
                                  torch.zeros(q9.shape[:3], device=DEV), None, 0)
 
 
+def test_decode_long_row_many_chunks_per_warp():
+    """A 90,000-slot row (one query head per KV head, the longest the logits buffer takes at this width): each
+    warp streams about 88 chunks, so its page ids come in three batches of 32."""
+    w = H.build(spec_of(Hq=1, Hkv=1, ctx=(90000,), seed=44, heavy=0.01))
+    q, q_pos = decode_inputs(w, q_pos=[70000])
+    scores = torch.zeros((w.spec.rows, w.spec.max_slots), device=DEV)
+    out, lse, status = run(w, q, q_pos, scores)
+    assert kvc.device_status(status)[0] == 0
+    check(w, q, q_pos, out, lse, scores, [0], "long row")
+
+
 def test_decode_full_size_sampled_rows():
     """The Llama-3-8B layer at 32K context, in the launch configuration the benchmark times
     (all 32 layers), checked on sampled rows."""
