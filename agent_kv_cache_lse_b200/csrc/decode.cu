@@ -70,6 +70,7 @@ struct DecodeShared {
     float pmax[kMaxGroup], psum[kMaxGroup];              // published CTA max and sum
     float pout[kMaxGroup * kMaxD];                       // published CTA output [g][d]
     float M[kMaxGroup], S[kMaxGroup];
+    float pw[kWarps][16 * kMaxGroup];                    // per-warp probabilities of a chunk [key][head]
     int32_t bad;
 };
 
@@ -115,6 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     constexpr int LK = D / 8;        // lanes per key
     constexpr int KW = 32 / LK;      // keys per warp step
     constexpr int MAXSTEPS = 16 / KW;
+    // reduce-scatter of the dot products when every lane can end with whole ones and the partials fit
+    constexpr bool kRS = MAXSTEPS * GM >= LK && MAXSTEPS * GM <= 32;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ DecodeShared sh;
     cg::cluster_group cl = cg::this_cluster();
@@ -225,17 +228,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         const T *Ks = reinterpret_cast<const T *>(ring + (size_t)st * stage_bytes);
         const T *Vs = Ks + CH * D;
         const int il0 = (warp + i * kWarps) * CH;
-        float l[MAXSTEPS][GM];
-        uint32_t vis = 0;
-        float cm[GM];
+        if constexpr (kRS) {
+            // the chunk's V = MAXSTEPS * GM partial dots per lane, reduced over the key's LK lanes by halving:
+            // lane sub ends with the R complete dots v = sub * R + r (step v / GM, head v % GM)
+            constexpr int V = MAXSTEPS * GM, R = V / LK;
+            float d[V];
+            uint32_t vis = 0;
 #pragma unroll
-        for (int g = 0; g < GM; ++g) cm[g] = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < MAXSTEPS; ++t) {
-            if (t < steps) {
+            for (int t = 0; t < MAXSTEPS; ++t) {
                 const int kk = t * KW + kslot;
-                const bool in = kk < CH && il0 + kk < cnt;
-                const bool v = page_ok && in && ps[il0 + kk] <= qpos;
+                const bool v = t < steps && page_ok && kk < CH && il0 + kk < cnt && ps[il0 + kk] <= qpos;
                 vis |= (v ? 1u : 0u) << t;
                 float2 x[4];
                 if (v) lds8(Ks + kk * D + sub * 8, x);
@@ -248,50 +250,160 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
                     acc = __ffma2_rn(qv[g][1], x[1], acc);
                     acc = __ffma2_rn(qv[g][2], x[2], acc);
                     acc = __ffma2_rn(qv[g][3], x[3], acc);
-                    float d = acc.x + acc.y;
-#pragma unroll
-                    for (int off = LK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-                    const float lv = v ? d * a.scale_log2 : -INFINITY;
-                    l[t][g] = lv;
-                    if (g < G && in && sub == 0) lg[(size_t)g * a.slice_cap + il0 + kk] = lv;
-                    cm[g] = fmaxf(cm[g], lv);
+                    d[t * GM + g] = acc.x + acc.y;
                 }
             }
-        }
 #pragma unroll
-        for (int g = 0; g < GM; ++g) {
+            for (int lvl = 0; (LK >> (lvl + 1)) > 0; ++lvl) {
+                const int off = LK >> (lvl + 1), n = V >> (lvl + 1);
+                const bool up = (sub & off) != 0;
 #pragma unroll
-            for (int off = LK; off < 32; off <<= 1) cm[g] = fmaxf(cm[g], __shfl_xor_sync(0xffffffffu, cm[g], off));
-            const float mn = fmaxf(m[g], cm[g]);
-            if (mn != m[g]) {  // warp-uniform: a new maximum rescales the running sum and output
-                const float f = weight(m[g], mn);
-                s[g] *= f;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) o[g][u] = __fmul2_rn(o[g][u], make_float2(f, f));
-                m[g] = mn;
+                for (int r = 0; r < n; ++r) {
+                    const float keep = up ? d[r + n] : d[r];
+                    const float send = up ? d[r] : d[r + n];
+                    d[r] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
             }
-        }
+            const int vbase = sub * R;
+            float lv[R];
+            float cm[GM];
 #pragma unroll
-        for (int t = 0; t < MAXSTEPS; ++t) {
-            if (t < steps && ((vis >> t) & 1u)) {
-                const int kk = t * KW + kslot;
-                float2 y[4];
-                lds8(Vs + kk * D + sub * 8, y);
+            for (int g = 0; g < GM; ++g) cm[g] = -INFINITY;
 #pragma unroll
-                for (int g = 0; g < GM; ++g) {
-                    const float p = ex2(l[t][g] - m[g]);
-                    s[g] += p;
+            for (int r = 0; r < R; ++r) {
+                const int v = vbase + r, t = v / GM, g = v % GM, kk = t * KW + kslot;
+                lv[r] = ((vis >> t) & 1u) ? d[r] * a.scale_log2 : -INFINITY;
+                if (g < G && t < steps && kk < CH && il0 + kk < cnt) lg[(size_t)g * a.slice_cap + il0 + kk] = lv[r];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) o[g][u] = __ffma2_rn(make_float2(p, p), y[u], o[g][u]);
+                for (int h = 0; h < GM; ++h)
+                    if (h == g) cm[h] = fmaxf(cm[h], lv[r]);
+            }
+#pragma unroll
+            for (int g = 0; g < GM; ++g) {
+                cm[g] = warp_max(cm[g]);
+                const float mn = fmaxf(m[g], cm[g]);
+                if (mn != m[g]) {  // warp-uniform: a new maximum rescales the running sums and output
+                    const float f = weight(m[g], mn);
+                    s[g] *= f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) o[g][u] = __fmul2_rn(o[g][u], make_float2(f, f));
+                    m[g] = mn;
+                }
+            }
+            // one exponential per (key, head); the key's lanes read all its heads' probabilities back
+            float *pwv = sh.pw[warp];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int v = vbase + r, t = v / GM, g = v % GM;
+                float mg = m[0];
+#pragma unroll
+                for (int h = 1; h < GM; ++h)
+                    if (h == g) mg = m[h];
+                const float p = lv[r] == -INFINITY ? 0.f : ex2(lv[r] - mg);
+#pragma unroll
+                for (int h = 0; h < GM; ++h)
+                    if (h == g) s[h] += p;
+                pwv[(t * KW + kslot) * GM + g] = p;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < MAXSTEPS; ++t) {
+                if ((vis >> t) & 1u) {
+                    const int kk = t * KW + kslot;
+                    float2 y[4];
+                    lds8(Vs + kk * D + sub * 8, y);
+                    float pp[GM];
+                    const float *src = pwv + kk * GM;
+                    if constexpr (GM % 4 == 0) {
+#pragma unroll
+                        for (int h = 0; h < GM; h += 4) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(src + h);
+                            pp[h] = f4.x; pp[h + 1] = f4.y; pp[h + 2] = f4.z; pp[h + 3] = f4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < GM; ++h) pp[h] = src[h];
+                    }
+#pragma unroll
+                    for (int g = 0; g < GM; ++g)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) o[g][u] = __ffma2_rn(make_float2(pp[g], pp[g]), y[u], o[g][u]);
+                }
+            }
+        } else {
+            float l[MAXSTEPS][GM];
+            uint32_t vis = 0;
+            float cm[GM];
+    #pragma unroll
+            for (int g = 0; g < GM; ++g) cm[g] = -INFINITY;
+    #pragma unroll
+            for (int t = 0; t < MAXSTEPS; ++t) {
+                if (t < steps) {
+                    const int kk = t * KW + kslot;
+                    const bool in = kk < CH && il0 + kk < cnt;
+                    const bool v = page_ok && in && ps[il0 + kk] <= qpos;
+                    vis |= (v ? 1u : 0u) << t;
+                    float2 x[4];
+                    if (v) lds8(Ks + kk * D + sub * 8, x);
+                    else
+    #pragma unroll
+                        for (int u = 0; u < 4; ++u) x[u] = make_float2(0.f, 0.f);
+    #pragma unroll
+                    for (int g = 0; g < GM; ++g) {
+                        float2 acc = __fmul2_rn(qv[g][0], x[0]);
+                        acc = __ffma2_rn(qv[g][1], x[1], acc);
+                        acc = __ffma2_rn(qv[g][2], x[2], acc);
+                        acc = __ffma2_rn(qv[g][3], x[3], acc);
+                        float d = acc.x + acc.y;
+    #pragma unroll
+                        for (int off = LK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                        const float lv = v ? d * a.scale_log2 : -INFINITY;
+                        l[t][g] = lv;
+                        if (g < G && in && sub == 0) lg[(size_t)g * a.slice_cap + il0 + kk] = lv;
+                        cm[g] = fmaxf(cm[g], lv);
+                    }
+                }
+            }
+    #pragma unroll
+            for (int g = 0; g < GM; ++g) {
+    #pragma unroll
+                for (int off = LK; off < 32; off <<= 1) cm[g] = fmaxf(cm[g], __shfl_xor_sync(0xffffffffu, cm[g], off));
+                const float mn = fmaxf(m[g], cm[g]);
+                if (mn != m[g]) {  // warp-uniform: a new maximum rescales the running sum and output
+                    const float f = weight(m[g], mn);
+                    s[g] *= f;
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) o[g][u] = __fmul2_rn(o[g][u], make_float2(f, f));
+                    m[g] = mn;
+                }
+            }
+    #pragma unroll
+            for (int t = 0; t < MAXSTEPS; ++t) {
+                if (t < steps && ((vis >> t) & 1u)) {
+                    const int kk = t * KW + kslot;
+                    float2 y[4];
+                    lds8(Vs + kk * D + sub * 8, y);
+    #pragma unroll
+                    for (int g = 0; g < GM; ++g) {
+                        const float p = ex2(l[t][g] - m[g]);
+                        s[g] += p;
+    #pragma unroll
+                        for (int u = 0; u < 4; ++u) o[g][u] = __ffma2_rn(make_float2(p, p), y[u], o[g][u]);
+                    }
                 }
             }
         }
         __syncwarp();  // every lane is done with stage st before the next issue refills it
     }
     cp_wait<0>();
-    // the warp's totals: sum over its key lanes (lanes that share sub)
+    // the warp's totals: the output over its key lanes (lanes that share sub); the sum over the lanes that
+    // hold distinct probabilities (all of them after the reduce-scatter, else one lane group per key)
 #pragma unroll
     for (int g = 0; g < GM; ++g) {
+        if constexpr (kRS) {
+#pragma unroll
+            for (int off = 1; off < LK; off <<= 1) s[g] += __shfl_xor_sync(0xffffffffu, s[g], off);
+        }
 #pragma unroll
         for (int off = LK; off < 32; off <<= 1) {
             s[g] += __shfl_xor_sync(0xffffffffu, s[g], off);
