@@ -319,14 +319,17 @@ def run_ours(args, rank, world, device):
 EvictionRound_KERNELS = 8
 
 SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_batch16_layer.md")
 
 
-def profiled_traffic():
-    """DRAM bytes per score_tc_kernel launch from the committed ncu summary, or None when the kernel source
-    has changed since those counters were taken (the summary records the source's sha256)."""
+def profiled_traffic(profile=None):
+    """DRAM bytes per launch of a kernel from its committed ncu summary (the scoring kernel's by default), or
+    None when the kernel source has changed since those counters were taken (the summary records the source's
+    sha256)."""
+    profile = profile or SCORE_PROFILE
     try:
         fields = {}
-        with open(SCORE_PROFILE) as f:
+        with open(profile) as f:
             for line in f:
                 if ":" in line and not line.startswith("#"):
                     k, _, v = line.partition(":")
@@ -592,7 +595,8 @@ def run_decode(args, device):
             "single_layer_32k": {"entries": entries1, "ms": ms1, "entries_per_s": entries1 / (ms1 / 1e3),
                                  "achieved_gbs": algo1 / (ms1 / 1e3) / 1e9},
             "roofline": {"kernel": "decode_kernel (kvc_decode_attention)", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": profiled_traffic(DECODE_PROFILE),
                          "peak_source": f"{kind} HBM copy", "bytes_per_launch": algo},
             "gpu_launches": args.steps}
 

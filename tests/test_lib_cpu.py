@@ -120,6 +120,30 @@ def test_bench_traffic_follows_kernel_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic() is None
     prof.write_text(f"source: {src}\nsource_sha256: {hashlib.sha256(b'x').hexdigest()}\ndram_bytes_per_launch: 5\n")
     assert bench.profiled_traffic() == 5
+    assert bench.profiled_traffic(str(prof)) == 5
+    d = bench.profiled_traffic(bench.DECODE_PROFILE)
+    assert d is None or d > 0
+
+
+def test_decode_host_validation_without_gpu():
+    """kvc_decode_attention refuses bad arguments, and rows whose logits cannot fit a cluster, before any launch
+    (the fake pointers are never dereferenced)."""
+    L = kvc.lib()
+    c = kvc.KvcCache()
+    c.num_seqs, c.num_layers, c.num_kv_heads = 1, 1, 1
+    c.page_size, c.max_pages_per_row, c.head_dim, c.dtype = 16, 4, 128, kvc.KVC_BF16
+    c.block_table = c.row_len = c.slot_pos = 256
+    c.k_pool = c.v_pool = 256
+    c.num_pages = 4
+    f = ctypes.c_void_p(256)
+    call = lambda q=f, hq=4, flags=0: L.kvc_decode_attention(ctypes.byref(c), q, f, hq, f, f, None, flags, None, None)
+    assert call(q=None) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert call(flags=2) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert call(hq=0) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert call(hq=9) == kvc.KVC_ERR_UNSUPPORTED            # 9 query heads per KV head
+    c.max_pages_per_row = 10000                             # 160,000 slots: logits beyond a cluster's memory
+    assert call() == kvc.KVC_ERR_UNSUPPORTED
+    assert b"logits" in L.kvc_last_error()
 
 
 def test_beacon_update_host_validation():
