@@ -299,6 +299,22 @@ kvc_status kvc_decode_attention(const kvc_cache *cache, const void *q, const int
                        "kvc_decode_attention launch");
 }
 
+kvc_status kvc_step_scores(const kvc_cache *cache, const float *scores, const int32_t *step_start,
+                           const int32_t *num_steps, int32_t max_steps, float beta, float *out, int32_t *d_status,
+                           kvc_stream_t stream) {
+    g_err[0] = 0;
+    kvc::CacheView c;
+    kvc_status s = view_cache(cache, c, false);
+    if (s != KVC_OK) return s;
+    if (!scores || !step_start || !num_steps || !out)
+        return fail(KVC_ERR_INVALID_ARGUMENT, "scores, step_start, num_steps and out are required");
+    if (max_steps < 1 || max_steps > 4096) return fail(KVC_ERR_UNSUPPORTED, "max_steps must be in [1, 4096]");
+    if (!(beta >= 0.f && beta <= 1.f)) return fail(KVC_ERR_INVALID_ARGUMENT, "beta must be in [0, 1]");
+    return cuda_status(kvc::launch_step_scores(c, scores, step_start, num_steps, max_steps, beta, out, d_status,
+                                               (cudaStream_t)stream),
+                       "kvc_step_scores launch");
+}
+
 kvc_status kvc_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params *params,
                             kvc_stream_t stream) {
     g_err[0] = 0;

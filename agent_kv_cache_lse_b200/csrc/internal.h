@@ -60,6 +60,9 @@ int decode_cluster(const CacheView &c, int32_t group);
 cudaError_t launch_decode(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                           float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream,
                           int cluster);
+cudaError_t launch_step_scores(const CacheView &c, const float *scores, const int32_t *step_start,
+                               const int32_t *num_steps, int32_t max_steps, float beta, float *out, int32_t *status,
+                               cudaStream_t stream);
 cudaError_t launch_ratchet_init(void *state, int32_t *budget, int32_t num_seqs, const kvc_ratchet_params &p,
                                 cudaStream_t stream);
 cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps, int32_t vocab, void *state,

@@ -23,12 +23,13 @@ KVC_F32, KVC_BF16 = 0, 1
 KVC_SCORE_ACCUMULATE, KVC_SCORE_COMPUTE_LSE, KVC_SCORE_SIMT = 1, 2, 4
 KVC_HIT_BINARY = 1
 DEV_CODES = {0: "ok", 1: "bad page", 2: "bad length", 3: "non-finite value", 4: "kept mismatch",
-             5: "freed list overflow", 6: "bad move", 7: "timeout"}
+             5: "freed list overflow", 6: "bad move", 7: "timeout", 8: "bad step table"}
 
 EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse", "kvc_score_from_lse",
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
-           "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select", "kvc_decode_attention"]
+           "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select", "kvc_decode_attention",
+           "kvc_step_scores"]
 
 
 class KvcCache(ctypes.Structure):
@@ -100,6 +101,7 @@ def lib() -> ctypes.CDLL:
             "kvc_beacon_update": (ctypes.c_int, [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp, vp, i32, vp, i32,
                                                  vp, vp]),
             "kvc_decode_attention": (ctypes.c_int, [pc, vp, vp, i32, vp, vp, vp, u32, vp, vp]),
+            "kvc_step_scores": (ctypes.c_int, [pc, vp, vp, vp, i32, f32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -286,6 +288,16 @@ def kvc_decode_attention(cache: Cache, q: torch.Tensor, q_pos: torch.Tensor, out
     _check(lib().kvc_decode_attention(ctypes.byref(cs), _ptr(q), _ptr(q_pos), q.shape[2], _ptr(out), _ptr(lse),
                                       _ptr(scores), flags, _ptr(d_status), _stream(stream)),
            "kvc_decode_attention")
+
+
+def kvc_step_scores(cache: Cache, scores: torch.Tensor, step_start: torch.Tensor, num_steps: torch.Tensor,
+                    out: torch.Tensor, beta: float = 0.5, d_status=None, stream=None):
+    """Step-aware ranking scores: (1 - beta) * s + beta * (mean score of the entry's step).  step_start:
+    [S][max_steps] int32 ascending from 0; num_steps: [S] int32; out: [rows][max_slots] fp32 (may be scores)."""
+    cs = cache.struct()
+    _check(lib().kvc_step_scores(ctypes.byref(cs), _ptr(scores), _ptr(step_start), _ptr(num_steps),
+                                 step_start.shape[1], beta, _ptr(out), _ptr(d_status), _stream(stream)),
+           "kvc_step_scores")
 
 
 def ratchet_seq_states(state: torch.Tensor, num_seqs: int):

@@ -242,6 +242,14 @@ def query_positions(spec: Spec, s: int) -> torch.Tensor:
     raise ValueError(spec.queries)
 
 
+def step_starts(spec: Spec, s: int) -> torch.Tensor:
+    """Start positions of the reasoning steps of sequence s: 0, then every position where a reasoning
+    segment begins (input construction for step-aware ranking; a ReAct step = thought, action, observation)."""
+    lab = segment_labels(spec, s, spec.ctx[s])
+    begin = torch.nonzero((lab[1:] == LABEL_REASON) & (lab[:-1] != LABEL_REASON)).flatten() + 1
+    return torch.cat([torch.zeros(1, dtype=torch.int64), begin]).to(torch.int32)
+
+
 # ----------------------------------------------------------------------------
 # paged layout and pools
 # ----------------------------------------------------------------------------

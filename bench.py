@@ -601,6 +601,58 @@ def run_decode(args, device):
             "gpu_launches": args.steps}
 
 
+def run_stepkv(args, device):
+    """Step-aware ranking scores (kvc_step_scores, beta 0.5) on the batch of 16 sequences x 8 layers x 8 KV heads
+    (context 8K-33K, step starts where reasoning segments begin): entries ranked per second, L2 flushed before
+    every call.  A separate line, not the eviction round."""
+    from agent_kv_cache_lse_b200 import kvc, synth
+    spec = synth.batch16(num_layers=8)
+    lay = synth.make_layout(spec)
+    starts = [synth.step_starts(spec, s) for s in range(spec.num_seqs)]
+    ms = max(len(x) for x in starts)
+    st = torch.full((spec.num_seqs, ms), 2**31 - 1, dtype=torch.int32)
+    for i, x in enumerate(starts):
+        st[i, :len(x)] = x
+    ns = torch.tensor([len(x) for x in starts], dtype=torch.int32, device=device)
+    st = st.to(device)
+    dummy = torch.zeros((1, 16, spec.head_dim), dtype=torch.bfloat16, device=device)
+    cache = kvc.Cache(dummy, dummy, lay.block_table.to(device), lay.row_len.to(device), lay.slot_pos.to(device),
+                      lay.slot_label.to(device), spec.num_seqs, spec.num_layers, spec.num_kv_heads)
+    gen = torch.Generator(device=device).manual_seed(5)
+    scores = torch.rand((spec.rows, spec.max_slots), generator=gen, device=device)
+    out = torch.empty_like(scores)
+    stt = torch.zeros(2, dtype=torch.int32, device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    for _ in range(max(3, args.warmup)):
+        kvc.kvc_step_scores(cache, scores, st, ns, out, 0.5, stt)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvc.kvc_step_scores(cache, scores, st, ns, out, 0.5, stt)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    assert int(stt[0]) == 0, kvc.device_status(stt)
+    entries = int(lay.row_len.sum())
+    algo = entries * 12 + spec.rows * 4 + spec.num_seqs * (ms + 1) * 4   # scores r, positions r, blend w
+    ms_ = float(np.median(ts))
+    hbm, _, _, kind = peaks()
+    achieved = algo / (ms_ / 1e3) / 1e9
+    return {"metric": "KV entries ranked/sec (step-aware scores)", "value": entries / (ms_ / 1e3), "unit": "entries/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"step-aware scores, batch of 16 sequences x 8 layers x 8 KV heads, context 8K-33K "
+                                   f"({entries} entries), {ms} steps at most per sequence, beta 0.5",
+                       "l2": "flushed (256 MB write) before every call"},
+            "roofline": {"kernel": "step_scores_kernel (kvc_step_scores)", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak_source": f"{kind} HBM copy", "bytes_per_launch": algo},
+            "gpu_launches": args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -611,6 +663,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
     ap.add_argument("--beacon", action="store_true", help="time beacon-query maintenance instead of the round")
     ap.add_argument("--decode", action="store_true", help="time the fused decode step instead of the round")
+    ap.add_argument("--stepkv", action="store_true", help="time the step-aware ranking scores instead of the round")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -630,6 +683,8 @@ def main():
         line = run_beacon(args, device)
     elif args.decode:
         line = run_decode(args, device)
+    elif args.stepkv:
+        line = run_stepkv(args, device)
     else:
         line = run_ours(args, rank, world, device)
     if world > 1:

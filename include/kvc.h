@@ -80,6 +80,7 @@ typedef enum {
 #define KVC_DEV_FREED_OVERFLOW 5 /* freed list longer than freed_capacity */
 #define KVC_DEV_BAD_MOVE 6       /* a move outside [0, row_len) or not hole/survivor */
 #define KVC_DEV_TIMEOUT 7        /* a bounded wait inside a kernel gave up */
+#define KVC_DEV_BAD_STEPS 8      /* step table not ascending from 0, num_steps out of range, or a negative position */
 
 typedef enum { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
 
@@ -370,6 +371,32 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
 kvc_status kvc_decode_attention(const kvc_cache *cache, const void *q, const int32_t *q_pos, int32_t num_q_heads,
                                 float *out, float *lse, float *scores, uint32_t flags, int32_t *d_status,
                                 kvc_stream_t stream);
+
+/*
+ * Step-aware ranking scores ("StepKV: Step-Aware KV Cache Compression for LLM Agents", abstract:
+ * entries belong to the reasoning step that generated them, a step utility from the trajectory is
+ * combined with token-level saliency, and the combined scores rank the prunable tokens under the
+ * budget).  The page gives no formulas; computed here, for every row and slot i < row_len:
+ *     step(i) = the last k with step_start[seq][k] <= slot_pos[i]
+ *     U_k     = mean of scores[row][i] over the row's slots of step k
+ *     out[row][i] = (1 - beta) * scores[row][i] + beta * U_step(i)
+ * The result ranks entries through kvc_select_budget (pass it as the crf argument), in place of
+ * or beside the LRFU values.
+ * scores:     [rows][max_slots] fp32 token saliency (e.g. the step-1 scores).
+ * step_start: [num_seqs][max_steps] int32 step start positions: step_start[s][0] = 0 and strictly
+ *             ascending over the first num_steps[s] entries (steps begin where reasoning segments
+ *             begin); a position maps to a step whatever slot the entry sits in, so the table
+ *             stays valid across compactions.
+ * num_steps:  [num_seqs] int32 in [1, max_steps].
+ * max_steps:  in [1, 4096]; beta in [0, 1].
+ * out:        [rows][max_slots] fp32, written for slots < row_len; may be the scores array itself.
+ * Step sums are exact integer sums of the scores rounded to a per-row fixed point (max|s| * 2^-39),
+ * so results repeat bit for bit.  d_status: KVC_DEV_BAD_STEPS, KVC_DEV_BAD_LENGTH, KVC_DEV_NONFINITE
+ * (the row is left unwritten).  One CTA per row.
+ */
+kvc_status kvc_step_scores(const kvc_cache *cache, const float *scores, const int32_t *step_start,
+                           const int32_t *num_steps, int32_t max_steps, float beta, float *out,
+                           int32_t *d_status, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -146,6 +146,30 @@ def test_decode_host_validation_without_gpu():
     assert b"logits" in L.kvc_last_error()
 
 
+def test_step_scores_host_validation_without_gpu():
+    """kvc_step_scores refuses bad arguments before any launch (fake pointers are never dereferenced)."""
+    L = kvc.lib()
+    c = kvc.KvcCache()
+    c.num_seqs, c.num_layers, c.num_kv_heads = 1, 1, 1
+    c.page_size, c.max_pages_per_row, c.head_dim, c.dtype = 16, 4, 128, kvc.KVC_BF16
+    c.block_table = c.row_len = c.slot_pos = 256
+    f = ctypes.c_void_p(256)
+    call = lambda sc=f, ms=8, beta=0.5: L.kvc_step_scores(ctypes.byref(c), sc, f, f, ms, ctypes.c_float(beta), f,
+                                                          None, None)
+    assert call(sc=None) == kvc.KVC_ERR_INVALID_ARGUMENT
+    assert call(ms=0) == kvc.KVC_ERR_UNSUPPORTED and call(ms=4097) == kvc.KVC_ERR_UNSUPPORTED
+    assert call(beta=1.5) == kvc.KVC_ERR_INVALID_ARGUMENT and call(beta=float("nan")) == kvc.KVC_ERR_INVALID_ARGUMENT
+
+
+def test_step_starts_follow_reasoning_segments():
+    spec = synth.llama8b_layer()
+    st = synth.step_starts(spec, 0).numpy()
+    lab = synth.segment_labels(spec, 0, spec.ctx[0]).numpy()
+    assert st[0] == 0 and np.all(np.diff(st) > 0)
+    assert np.all(lab[st[1:]] == synth.LABEL_REASON) and np.all(lab[st[1:] - 1] != synth.LABEL_REASON)
+    assert len(st) - 1 == int(((lab[1:] == synth.LABEL_REASON) & (lab[:-1] != synth.LABEL_REASON)).sum())
+
+
 def test_beacon_update_host_validation():
     """Bad sizes are refused before anything reaches the device (fake pointers are never dereferenced)."""
     from agent_kv_cache_lse_b200 import kvc
