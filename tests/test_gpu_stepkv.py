@@ -92,11 +92,12 @@ def test_beta_zero_is_the_saliency_and_in_place_is_the_same():
 
 
 def test_bad_step_tables_are_reported():
-    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=(600, 700), L=1, Hkv=2, seed=53)
+    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=(5000, 6000), L=1, Hkv=2, seed=53)
+    assert int(ns[1]) >= 2, "the case needs two steps in sequence 1"
     out = torch.zeros_like(s)
     status = torch.zeros(2, dtype=torch.int32, device=DEV)
     st2 = st.clone()
-    st2[1, 1] = st2[1, 2]                                   # not strictly ascending in sequence 1
+    st2[1, 1] = st2[1, 0]                                   # not strictly ascending in sequence 1
     kvc.kvc_step_scores(cache, s, st2, ns, out, 0.5, status)
     torch.cuda.synchronize()
     code, row, _ = kvc.device_status(status)
