@@ -11,7 +11,9 @@
 //   out[i]   = (1 - beta) * s[i] + beta * U_step(i).
 // The output feeds the same top-budget selection as the LRFU values.
 //
-// One CTA per row.  Pass 1 finds max |s| of the row, which fixes a power-of-two scale; pass 2
+// One CTA per row.  Rows of up to 34,816 slots keep their scores in registers (1,024 threads x 34) and
+// their step ids in shared memory, so scores and positions are read once; longer rows take three passes
+// over global memory.  Pass 1 finds max |s| of the row, which fixes a power-of-two scale; pass 2
 // adds every score, rounded to a 64-bit fixed-point integer at that scale, into its step's sum in
 // shared memory (integer adds, so the sums do not depend on the order of the atomics; a warp whose
 // lanes share a step adds once); pass 3 writes the blend.  The fixed point carries each score to
@@ -142,11 +144,134 @@ __global__ void __launch_bounds__(kThreads) step_scores_kernel(StepArgs a) {
     }
 }
 
+// Rows of at most kRegThreads * kRegSlots slots: each thread keeps its slots' scores in registers and their
+// step ids in shared memory, so the row's scores and positions are read from HBM once.
+constexpr int kRegThreads = 1024;
+constexpr int kRegSlots = 34;  // 34,816 slots: the 33K-token rows of the workloads
+
+__global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int row = blockIdx.x;
+    const CacheView &c = a.c;
+    const int seq = row / (c.num_layers * c.num_kv_heads);
+    int64_t *sum = reinterpret_cast<int64_t *>(smem);                    // [max_steps]
+    int32_t *cnt = reinterpret_cast<int32_t *>(sum + a.max_steps);        // [max_steps]
+    int32_t *starts = cnt + a.max_steps;                                  // [max_steps]
+    uint16_t *sid = reinterpret_cast<uint16_t *>(starts + a.max_steps);  // [kRegThreads * kRegSlots] step ids
+    __shared__ float red[kRegThreads / 32];
+    __shared__ int bad;
+    const int tid = threadIdx.x, lane = tid & 31;
+
+    const int n = c.row_len[row];
+    const int ns = a.num_steps[seq];
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    if (ns < 1 || ns > a.max_steps) {
+        if (tid == 0) report(a.status, KVC_DEV_BAD_STEPS, row);
+        return;
+    }
+    if (n < 0 || n > c.max_slots) {
+        if (tid == 0) report(a.status, KVC_DEV_BAD_LENGTH, row);
+        return;
+    }
+    const int32_t *st = a.step_start + (int64_t)seq * a.max_steps;
+    for (int k = tid; k < ns; k += kRegThreads) {
+        const int32_t v = st[k];
+        starts[k] = v;
+        sum[k] = 0;
+        cnt[k] = 0;
+        if ((k == 0 && v != 0) || (k > 0 && v <= st[k - 1])) bad = 1;
+    }
+    const float *s = a.scores + (int64_t)row * c.max_slots;
+    const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots;
+    float v[kRegSlots];
+#pragma unroll
+    for (int j = 0; j < kRegSlots; ++j) {  // the row's scores, all loads in flight together
+        const int i = tid + j * kRegThreads;
+        v[j] = i < n ? s[i] : 0.f;
+    }
+    __syncthreads();  // the step table is in place
+    constexpr int kPart = 8;
+#pragma unroll
+    for (int h = 0; h < (kRegSlots + kPart - 1) / kPart; ++h) {  // positions in parts, to stay within the registers
+        int32_t p[kPart];
+#pragma unroll
+        for (int j = 0; j < kPart; ++j) {
+            const int i = tid + (h * kPart + j) * kRegThreads;
+            p[j] = (h * kPart + j < kRegSlots && i < n) ? pos[i] : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < kPart; ++j) {
+            const int i = tid + (h * kPart + j) * kRegThreads;
+            if (h * kPart + j < kRegSlots && i < n) {
+                if (p[j] < 0) bad = 1;
+                else sid[i] = (uint16_t)step_of(starts, ns, p[j]);
+            }
+        }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < kRegSlots; ++j) mx = fmaxf(mx, fabsf(v[j]));
+    mx = block_max(mx, red);
+    if (bad || !is_finite(mx)) {
+        if (tid == 0) report(a.status, bad ? KVC_DEV_BAD_STEPS : KVC_DEV_NONFINITE, row);
+        return;
+    }
+    int e = 0;
+    if (mx > 0.f) frexpf(mx, &e);
+    const double scale = ldexp(1.0, 39 - e);
+#pragma unroll
+    for (int j = 0; j < kRegSlots; ++j) {
+        const int i = tid + j * kRegThreads;
+        if (j * kRegThreads >= n) break;  // block-uniform
+        const bool in = i < n;
+        const int k = in ? sid[i] : 0;
+        const long long qv = in ? __double2ll_rn((double)v[j] * scale) : 0;
+        const unsigned vm = __ballot_sync(0xffffffffu, in);
+        const int k0 = __shfl_sync(0xffffffffu, k, 0);
+        if (vm == 0xffffffffu && __all_sync(0xffffffffu, k == k0)) {
+            long long t = qv;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+            if (lane == 0) {
+                atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k0]), (unsigned long long)t);
+                atomicAdd(&cnt[k0], 32);
+            }
+        } else if (in) {
+            atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k]), (unsigned long long)qv);
+            atomicAdd(&cnt[k], 1);
+        }
+    }
+    __syncthreads();
+    double *u = reinterpret_cast<double *>(sum);
+    for (int k = tid; k < ns; k += kRegThreads) {
+        const long long t = sum[k];
+        u[k] = cnt[k] > 0 ? (double)t / (scale * (double)cnt[k]) : 0.0;
+    }
+    __syncthreads();
+    float *o = a.out + (int64_t)row * c.max_slots;
+    const float w = 1.f - a.beta;
+#pragma unroll
+    for (int j = 0; j < kRegSlots; ++j) {
+        const int i = tid + j * kRegThreads;
+        if (i < n) o[i] = fmaf(a.beta, (float)u[sid[i]], w * v[j]);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_step_scores(const CacheView &c, const float *scores, const int32_t *step_start,
                                const int32_t *num_steps, int32_t max_steps, float beta, float *out, int32_t *status,
                                cudaStream_t stream) {
+    if (c.max_slots <= (int64_t)kRegThreads * kRegSlots && max_steps <= 65536) {
+        const size_t smem = (size_t)max_steps * (8 + 4 + 4) + (size_t)kRegThreads * kRegSlots * 2;
+        cudaError_t e = cudaFuncSetAttribute(step_scores_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        step_scores_reg_kernel<<<c.rows, kRegThreads, smem, stream>>>(
+            StepArgs{c, scores, step_start, num_steps, max_steps, beta, out, status});
+        return cudaGetLastError();
+    }
     const size_t smem = (size_t)max_steps * (8 + 4 + 4);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(step_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

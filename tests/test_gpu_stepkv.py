@@ -55,10 +55,12 @@ def check(spec, out, sc, pos, rl, starts, beta, what):
         assert not bad.any(), f"{what} row {r}: {int(bad.sum())} values out of tolerance, max err {err.max()}"
 
 
-@pytest.mark.parametrize("case", ["plain", "permuted_short", "beta03", "beta1"])
+@pytest.mark.parametrize("case", ["plain", "permuted_short", "beta03", "beta1", "long_rows"])
 def test_step_scores_parity(case):
+    """Rows up to 34,816 slots run the register-resident kernel; "long_rows" (40,000 slots) the three-pass one."""
     beta = {"beta03": 0.3, "beta1": 1.0}.get(case, 0.5)
-    spec, cache, s, st, ns, sc, pos, rl, starts = workload(permute=case == "permuted_short",
+    ctx = (40000, 1200) if case == "long_rows" else (1500, 2817, 4000)
+    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=ctx, permute=case in ("permuted_short", "long_rows"),
                                                            shorten=case == "permuted_short")
     out = torch.full_like(s, -5.0)
     status = torch.zeros(2, dtype=torch.int32, device=DEV)
