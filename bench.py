@@ -320,6 +320,7 @@ EvictionRound_KERNELS = 8
 
 SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_batch16_layer.md")
+STEPKV_PROFILE = os.path.join(ROOT, "profiles", "step_scores_batch16_8layers.md")
 
 
 def profiled_traffic(profile=None):
@@ -647,8 +648,9 @@ def run_stepkv(args, device):
             "config": {"workload": f"step-aware scores, batch of 16 sequences x 8 layers x 8 KV heads, context 8K-33K "
                                    f"({entries} entries), {ms} steps at most per sequence, beta 0.5",
                        "l2": "flushed (256 MB write) before every call"},
-            "roofline": {"kernel": "step_scores_kernel (kvc_step_scores)", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+            "roofline": {"kernel": "step_scores_reg_kernel (kvc_step_scores)", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": profiled_traffic(STEPKV_PROFILE),
                          "peak_source": f"{kind} HBM copy", "bytes_per_launch": algo},
             "gpu_launches": args.steps}
 
