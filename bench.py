@@ -11,6 +11,13 @@ write) outside the timed region before every step.
 
 Prints one JSON line (rank 0).  N > 1 runs one independent replica per GPU (weak scaling:
 the path shards by sequence and needs no collective).
+
+Separate single-GPU lines for the entry points beside the round, each with its own workload,
+metric and roofline:
+  --decode   one decode step of paged attention with the scores folded in (kvc_decode_attention),
+             one layer of the batch of 16 sequences at 8K-33K;
+  --stepkv   step-aware ranking scores (kvc_step_scores), 16 sequences x 8 layers x 8 KV heads;
+  --beacon   beacon-query maintenance (kvc_beacon_update), the streaming shape.
 """
 from __future__ import annotations
 
