@@ -127,6 +127,16 @@ def _check(status: int, what: str):
         raise KvcError(f"{what}: {L.kvc_status_string(status).decode()}: {L.kvc_last_error().decode()}")
 
 
+def _expect(t: torch.Tensor, name: str, shape, dtype):
+    """Raise KvcError unless t is a contiguous tensor of the given dtype and shape (None = any extent)."""
+    if t.dtype != dtype:
+        raise KvcError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.dim() != len(shape) or any(e is not None and t.shape[i] != e for i, e in enumerate(shape)):
+        raise KvcError(f"{name}: shape {tuple(t.shape)}, expected {tuple('*' if e is None else e for e in shape)}")
+    if not t.is_contiguous():
+        raise KvcError(f"{name} must be contiguous")
+
+
 @dataclass
 class Cache:
     """Device tensors of a paged cache (see kvc_cache in include/kvc.h)."""
@@ -283,7 +293,15 @@ def kvc_decode_attention(cache: Cache, q: torch.Tensor, q_pos: torch.Tensor, out
                          scores: Optional[torch.Tensor] = None, flags: int = 0, d_status=None, stream=None):
     """One decode step with the scores folded in.  q: [S][L][Hq][D] in the cache dtype; q_pos: [S] int32;
     out: [S][L][Hq][D] fp32; lse: [S][L][Hq] fp32; scores: optional [rows][max_slots] fp32
-    (KVC_SCORE_ACCUMULATE adds into it)."""
+    (KVC_SCORE_ACCUMULATE adds into it).  Shapes and dtypes, which the C ABI cannot see, are checked here."""
+    S, L, D = cache.num_seqs, cache.num_layers, cache.k_pool.shape[2]
+    _expect(q, "q", (S, L, None, D), cache.k_pool.dtype)
+    Hq = q.shape[2]
+    _expect(q_pos, "q_pos", (S,), torch.int32)
+    _expect(out, "out", (S, L, Hq, D), torch.float32)
+    _expect(lse, "lse", (S, L, Hq), torch.float32)
+    if scores is not None:
+        _expect(scores, "scores", (cache.rows, cache.max_slots), torch.float32)
     cs = cache.struct()
     _check(lib().kvc_decode_attention(ctypes.byref(cs), _ptr(q), _ptr(q_pos), q.shape[2], _ptr(out), _ptr(lse),
                                       _ptr(scores), flags, _ptr(d_status), _stream(stream)),
@@ -294,6 +312,10 @@ def kvc_step_scores(cache: Cache, scores: torch.Tensor, step_start: torch.Tensor
                     out: torch.Tensor, beta: float = 0.5, d_status=None, stream=None):
     """Step-aware ranking scores: (1 - beta) * s + beta * (mean score of the entry's step).  step_start:
     [S][max_steps] int32 ascending from 0; num_steps: [S] int32; out: [rows][max_slots] fp32 (may be scores)."""
+    _expect(scores, "scores", (cache.rows, cache.max_slots), torch.float32)
+    _expect(out, "out", (cache.rows, cache.max_slots), torch.float32)
+    _expect(step_start, "step_start", (cache.num_seqs, None), torch.int32)
+    _expect(num_steps, "num_steps", (cache.num_seqs,), torch.int32)
     cs = cache.struct()
     _check(lib().kvc_step_scores(ctypes.byref(cs), _ptr(scores), _ptr(step_start), _ptr(num_steps),
                                  step_start.shape[1], beta, _ptr(out), _ptr(d_status), _stream(stream)),

@@ -170,6 +170,32 @@ def test_step_starts_follow_reasoning_segments():
     assert len(st) - 1 == int(((lab[1:] == synth.LABEL_REASON) & (lab[:-1] != synth.LABEL_REASON)).sum())
 
 
+def test_binding_checks_shapes_and_dtypes():
+    """The Python binding refuses mismatched tensors before the C call (CPU tensors: nothing reaches a device)."""
+    S, L, Hkv, P, D, mp = 2, 1, 2, 16, 64, 4
+    rows = S * L * Hkv
+    cache = kvc.Cache(torch.zeros((8, P, D), dtype=torch.bfloat16), torch.zeros((8, P, D), dtype=torch.bfloat16),
+                      torch.zeros((rows, mp), dtype=torch.int32), torch.zeros(rows, dtype=torch.int32),
+                      torch.zeros((rows, mp * P), dtype=torch.int32), None, S, L, Hkv)
+    q = torch.zeros((S, L, 4, D), dtype=torch.bfloat16)
+    qp = torch.zeros(S, dtype=torch.int32)
+    out, lse = torch.zeros((S, L, 4, D)), torch.zeros((S, L, 4))
+    with pytest.raises(kvc.KvcError, match="q: dtype"):
+        kvc.kvc_decode_attention(cache, q.float(), qp, out, lse)
+    with pytest.raises(kvc.KvcError, match="out: shape"):
+        kvc.kvc_decode_attention(cache, q, qp, out[:, :, :2], lse)
+    with pytest.raises(kvc.KvcError, match="scores: shape"):
+        kvc.kvc_decode_attention(cache, q, qp, out, lse, torch.zeros((rows, 5)))
+    with pytest.raises(kvc.KvcError, match="q_pos: dtype"):
+        kvc.kvc_decode_attention(cache, q, qp.long(), out, lse)
+    sc = torch.zeros((rows, mp * P))
+    st, ns = torch.zeros((S, 3), dtype=torch.int32), torch.ones(S, dtype=torch.int32)
+    with pytest.raises(kvc.KvcError, match="step_start: shape"):
+        kvc.kvc_step_scores(cache, sc, st[:1], ns, sc)
+    with pytest.raises(kvc.KvcError, match="out must be contiguous"):
+        kvc.kvc_step_scores(cache, sc, st, ns, torch.zeros((mp * P, rows)).t())
+
+
 def test_beacon_update_host_validation():
     """Bad sizes are refused before anything reaches the device (fake pointers are never dereferenced)."""
     from agent_kv_cache_lse_b200 import kvc
