@@ -392,7 +392,8 @@ kvc_status kvc_decode_attention(const kvc_cache *cache, const void *q, const int
  * out:        [rows][max_slots] fp32, written for slots < row_len; may be the scores array itself.
  * Step sums are exact integer sums of the scores rounded to a per-row fixed point (max|s| * 2^-39),
  * so results repeat bit for bit.  d_status: KVC_DEV_BAD_STEPS, KVC_DEV_BAD_LENGTH, KVC_DEV_NONFINITE
- * (the row is left unwritten).  One CTA per row.
+ * for an infinite score (the row is left unwritten); a NaN score is not detected and leaves the
+ * row's results undefined.  One CTA per row.
  */
 kvc_status kvc_step_scores(const kvc_cache *cache, const float *scores, const int32_t *step_start,
                            const int32_t *num_steps, int32_t max_steps, float beta, float *out,

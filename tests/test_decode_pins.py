@@ -54,6 +54,18 @@ def test_no_visible_key():
     assert np.all(np.isneginf(lse)) and np.all(out == 0) and np.all(inc == 0)
 
 
+def test_increment_agrees_with_the_scoring_oracle():
+    """One decode query's score increment is the scoring step's per-query term: the decode oracle (output path)
+    and the scoring oracle (exp(logit - lse) summed over the group) agree on the same query and LSE."""
+    from oracle import path as op
+    rng = np.random.default_rng(7)
+    q, k, v, pos = _case(rng, G=3, n=250)
+    qpos = int(np.sort(pos)[180])
+    out, lse, inc = od.decode_step(q, k, v, qpos, pos)
+    s = op.scores_from_lse(q[None], k, np.array([qpos]), pos, lse[:, None])
+    assert np.allclose(inc, s, rtol=1e-12, atol=1e-15)
+
+
 @pytest.mark.parametrize("mistake", ["no_scale", "mask_reversed", "unnormalised"])
 def test_planted_mistakes_are_caught(mistake, monkeypatch):
     from oracle import path as op
