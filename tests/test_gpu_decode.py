@@ -215,3 +215,15 @@ def test_decode_full_size_sampled_rows():
     # every row's scores sum to its group size (the probabilities of each head sum to one)
     sums = scores.sum(dim=1).cpu().numpy()
     assert np.all(np.abs(sums - spec.group) <= 1e-3 * spec.group)
+
+
+def test_decode_bench_workload_sampled_rows():
+    """The workload and launch configuration bench.py --decode times: one layer of the batch of 16 sequences
+    (context 8K-33K, 128 rows, clusters of 8), checked on sampled rows."""
+    spec = synth.batch16(num_layers=1)
+    w = H.build(spec)
+    q, q_pos = decode_inputs(w)
+    scores = torch.zeros((spec.rows, spec.max_slots), device=DEV)
+    out, lse, status = run(w, q, q_pos, scores, kvc.KVC_SCORE_ACCUMULATE)
+    assert kvc.device_status(status)[0] == 0
+    check(w, q, q_pos, out, lse, scores, [0, 37, 64, 101, 127], "batch16 layer")

@@ -136,3 +136,22 @@ def test_selection_on_step_scores_matches_the_oracle():
         assert int(kept[r]) == min(700, n)
         # and the GPU's own selection is exact on its own blended values
         assert np.array_equal(k[r, :n], opath.select_budget(o[r, :n].astype(np.float64), pos[r, :n], 700))
+
+
+def test_step_scores_bench_workload_sampled_rows():
+    """The workload bench.py --stepkv times: 16 sequences x 8 layers x 8 KV heads at 8K-33K (1,024 rows, the
+    register-resident kernel), checked on sampled rows."""
+    b = synth.batch16(num_layers=8)
+    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=tuple(b.ctx), L=8, Hkv=8, seed=55)
+    out = torch.zeros_like(s)
+    status = torch.zeros(2, dtype=torch.int32, device=DEV)
+    kvc.kvc_step_scores(cache, s, st, ns, out, 0.5, status)
+    torch.cuda.synchronize()
+    assert kvc.device_status(status)[0] == 0
+    got = out.cpu().numpy()
+    for r in (0, 255, 511, 800, 1023):
+        s_, _, _ = spec.row_coords(r)
+        n = int(rl[r])
+        want = osk.combined_scores(sc[r, :n].astype(np.float64), pos[r, :n], starts[s_].numpy(), 0.5)
+        err = np.abs(got[r, :n] - want)
+        assert np.all(err <= 1e-6 + 1e-3 * np.abs(want)), f"row {r}: max err {err.max()}"
