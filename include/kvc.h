@@ -358,11 +358,13 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
  * scores:  NULL (attention only) or [rows][max_pages_per_row * page_size] fp32, written
  *          (added to with KVC_SCORE_ACCUMULATE) for slots < row_len only.
  * flags:   0 or KVC_SCORE_ACCUMULATE.
- * Limits:  num_q_heads / num_kv_heads <= 8, and a CTA of the row's cluster (at most 8 CTAs)
- *          must hold its slice's logits and positions, (G' + 1) * 4 * ceil(max_slots / 8) bytes
- *          (G' = the group size rounded up to a power of two), beside two K/V stages per warp of
- *          a chunk (up to 16 slots of one page), within 220 KiB: for bf16 and head_dim
- *          128, max_slots up to about 37,000 at G = 4 and 94,000 at G = 1; otherwise
+ * Limits:  num_q_heads / num_kv_heads <= 8.  Each CTA of the row's cluster (at most 8 CTAs) keeps
+ *          its slice's logits and positions, (G' + 1) * 4 * ceil(max_slots / 8) bytes (G' = the
+ *          group size rounded up to a power of two), beside at least two K/V stages per warp, all
+ *          within 220 KiB; a stage holds a chunk of 16 slots of one page, shrinking to 8, 4, 2 or 1
+ *          slots (slower) when 16 do not fit.  For bf16 and head_dim 128, 16-slot chunks serve rows
+ *          up to 94,208 / 62,720 / 37,632 / 20,864 slots at G = 1 / 2 / 4 / 8, and the longest rows
+ *          accepted are 217,088 / 144,720 / 83,552 / 42,768 slots; longer ones return
  *          KVC_ERR_UNSUPPORTED.  d_status reports a bad page or a bad row length; the affected
  *          row's results are then undefined.
  * Every sum runs in a fixed order: results repeat bit for bit.  One cluster of up to 8 CTAs

@@ -146,6 +146,25 @@ def test_decode_host_validation_without_gpu():
     assert b"logits" in L.kvc_last_error()
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="a supported size would launch the kernel on fake pointers")
+@pytest.mark.parametrize("group,limit", [(1, 217088), (2, 144720), (4, 83552), (8, 42768)])
+def test_decode_row_limit_matches_the_header(group, limit):
+    """bf16, head_dim 128, 16-slot pages: the longest row the decode entry point takes, as the header states it.
+    Without a GPU a supported size gets as far as the launch and fails there (KVC_ERR_CUDA); one page more is
+    refused on the host (KVC_ERR_UNSUPPORTED)."""
+    L = kvc.lib()
+    c = kvc.KvcCache()
+    c.num_seqs, c.num_layers, c.num_kv_heads = 1, 1, 8
+    c.page_size, c.head_dim, c.dtype = 16, 128, kvc.KVC_BF16
+    c.block_table = c.row_len = c.slot_pos = 256
+    c.k_pool = c.v_pool = 256
+    c.num_pages = 4
+    f = ctypes.c_void_p(256)
+    for pages, want in ((limit // 16, kvc.KVC_ERR_CUDA), (limit // 16 + 1, kvc.KVC_ERR_UNSUPPORTED)):
+        c.max_pages_per_row = pages
+        assert L.kvc_decode_attention(ctypes.byref(c), f, f, 8 * group, f, f, f, 0, None, None) == want, pages
+
+
 def test_step_scores_host_validation_without_gpu():
     """kvc_step_scores refuses bad arguments before any launch (fake pointers are never dereferenced)."""
     L = kvc.lib()
