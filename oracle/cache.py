@@ -8,6 +8,11 @@ TEST INFRASTRUCTURE ONLY (see ``oracle.path``).  Layouts, all host numpy arrays:
 * ``block_table``: [rows, max_pages], -1 = no page; row = (seq * layers + layer) * kv_heads + head.
 * ``row_len``: [rows]; ``slot_pos``/``slot_label``: [rows, max_pages * page_size].
 * queries: ``q`` [S, L, max_q, Hq, D], ``lse`` [S, L, Hq, max_q], ``q_pos`` [S, max_q], ``num_q`` [S].
+
+Parity status: pinned on a hand-built, permuted cache by the non-GPU tests (row-id order,
+gathers against per-slot identity codes, LSE and scores by brute force, the per-row steps
+against the pinned ``oracle.path`` functions, compaction against a written-out single copy
+pass and the freed-list order), with planted mistakes that must each fail a pin.
 """
 from __future__ import annotations
 
