@@ -40,6 +40,12 @@ __device__ __forceinline__ bool row_ok(const CacheView &c, int n, int m) {
     return n >= 0 && n <= c.max_slots && m >= 0 && m <= n;
 }
 
+// A row is compacted only when its lengths and its move count are consistent; any other row (among
+// them the rows the planner rejected, num_moves = -1) keeps its pages, block table and row_len.
+__device__ __forceinline__ bool row_plan_ok(const CacheView &c, int n, int m, int nm) {
+    return row_ok(c, n, m) && nm >= 0 && nm <= m && nm <= n - m;
+}
+
 __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 __device__ void freed_offsets(const CompactArgs &a) {
@@ -53,7 +59,7 @@ __device__ void freed_offsets(const CompactArgs &a) {
         int f = 0;
         if (r < c.rows) {
             const int n = c.row_len[r], m = a.new_len[r];
-            if (row_ok(c, n, m)) f = (int)(ceil_div(n, c.page_size) - ceil_div(m, c.page_size));
+            if (row_plan_ok(c, n, m, a.num_moves[r])) f = (int)(ceil_div(n, c.page_size) - ceil_div(m, c.page_size));
         }
         int total;
         const int ex = block_exclusive_scan(f, red, &total);
@@ -79,8 +85,9 @@ __global__ void __launch_bounds__(kThreads) compact_moves_kernel(CompactArgs a) 
     const int row = blockIdx.y;
     const int n = c.row_len[row], m = a.new_len[row];
     const int nm = a.num_moves[row];
-    if (!row_ok(c, n, m) || nm < 0 || nm > m || nm > n - m) {
-        if (blockIdx.x == 0 && threadIdx.x == 0)
+    if (!row_plan_ok(c, n, m, nm)) {
+        // num_moves = -1: the planner rejected the row and has reported why
+        if (blockIdx.x == 0 && threadIdx.x == 0 && nm != -1)
             report(a.status, row_ok(c, n, m) ? KVC_DEV_BAD_MOVE : KVC_DEV_BAD_LENGTH, row);
         return;
     }
@@ -120,7 +127,7 @@ __global__ void __launch_bounds__(kThreads) compact_free_kernel(CompactArgs a) {
     const CacheView &c = a.c;
     const int row = blockIdx.y;
     const int n = c.row_len[row], m = a.new_len[row];
-    if (!row_ok(c, n, m)) return;
+    if (!row_plan_ok(c, n, m, a.num_moves[row])) return;
     const int64_t first = ceil_div(m, c.page_size), end = ceil_div(n, c.page_size);
     const int64_t base = a.row_offsets[row];
     // all of a row's pages go back, or (when the list is too short) none of them

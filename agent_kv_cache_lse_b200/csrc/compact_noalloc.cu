@@ -1,9 +1,8 @@
 // kvc_compact_pages_noalloc: the compaction entry point for callers that cannot allocate.
 //
 // kvc_compact_pages needs a small device workspace (one 64-bit offset per row) for the
-// freed-page list.  Some callers have no way to provide one: code that runs while a
-// CUDA graph is being captured (a cudaMalloc there breaks the capture), serving engines
-// whose allocator has already handed the whole device to the KV pool, or plugins that
+// freed-page list.  Some callers have no way to provide one: serving engines whose
+// allocator has already handed the whole device to the KV pool, or plugins that
 // reach this library through a foreign-function boundary without access to the host
 // framework's allocator.  This variant keeps the workspace in a fixed array in the
 // library's own device memory instead, so the caller passes only the cache, the plan

@@ -35,9 +35,10 @@ __global__ void __launch_bounds__(kThreads) plan_kernel(PlanArgs a) {
     const CacheView &c = a.c;
     const int n = c.row_len[row];
     const int m = a.kept[row];
+    // A rejected row gets num_moves = -1, which the compaction reads as "leave this row as it is".
     if (n < 0 || n > c.max_slots || m < 0 || m > n) {
         if (rc.rank == 0 && threadIdx.x == 0) {
-            a.num_moves[row] = 0;
+            a.num_moves[row] = -1;
             report(a.status, (n < 0 || n > c.max_slots) ? KVC_DEV_BAD_LENGTH : KVC_DEV_KEPT_MISMATCH, row);
         }
         return;
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) plan_kernel(PlanArgs a) {
     // kept count consistent with the mask  <=>  as many holes before m as survivors after it
     if (tot[0] != tot[1]) {
         if (rc.rank == 0 && threadIdx.x == 0) {
-            a.num_moves[row] = 0;
+            a.num_moves[row] = -1;
             report(a.status, KVC_DEV_KEPT_MISMATCH, row);
         }
         rc.cl.sync();

@@ -245,7 +245,7 @@ def kvc_compact_pages(cache: Cache, move_src, move_dst, num_moves, new_len, crf:
 def kvc_compact_pages_noalloc(cache: Cache, move_src, move_dst, num_moves, new_len, crf: Optional[torch.Tensor],
                               freed: torch.Tensor, num_freed: torch.Tensor, d_status=None, stream=None):
     """kvc_compact_pages with the library's built-in workspace, for callers that cannot allocate device memory
-    (e.g. during CUDA graph capture, or when the KV pool owns all free memory).  At most KVC_NOALLOC_MAX_ROWS
+    (e.g. when the KV pool owns all free memory, or behind a foreign-function boundary).  At most KVC_NOALLOC_MAX_ROWS
     rows; calls that overlap on the GPU share the workspace and must be serialised."""
     cs = cache.struct()
     _check(lib().kvc_compact_pages_noalloc(ctypes.byref(cs), _ptr(move_src), _ptr(move_dst), _ptr(num_moves),

@@ -237,6 +237,10 @@ kvc_status kvc_lrfu_select(const kvc_cache *cache, const float *scores, float *c
  * survivors are the slots i >= m with keep 1, both ascending; move j copies survivor j
  * into hole j.  move_src/move_dst: [rows][max_slots] int32 (first num_moves[row] valid).
  * No slot is written twice and no destination is a source, so one parallel pass is safe.
+ * A row whose kept count disagrees with its mask (as many holes before m as survivors
+ * after it is the condition), or whose row_len is out of range, is reported in d_status
+ * (KVC_DEV_KEPT_MISMATCH / KVC_DEV_BAD_LENGTH) and gets num_moves[row] = -1; the
+ * compaction leaves such a row exactly as it is.
  */
 kvc_status kvc_plan_slots(const kvc_cache *cache, const uint8_t *keep, const int32_t *kept,
                           int32_t *move_src, int32_t *move_dst, int32_t *num_moves,
@@ -254,6 +258,13 @@ size_t kvc_compact_workspace_bytes(int32_t rows);
  * freed: [freed_capacity] int32; *num_freed (device int64) = total freed.  Source slots
  * are not cleared.  workspace: at least kvc_compact_workspace_bytes(rows) bytes of
  * device memory whose contents need not be preserved between calls.
+ * A row is compacted only when 0 <= new_len <= row_len <= max_slots and
+ * 0 <= num_moves <= min(new_len, row_len - new_len); any other row (num_moves = -1 from
+ * the planner included) keeps its pool bytes, block table, positions and row_len.
+ * Freed-list overflow (KVC_DEV_FREED_OVERFLOW): *num_freed is the total the list would
+ * need, so it can exceed freed_capacity; the rows whose pages fit are listed as usual;
+ * a row whose pages do not all fit lists none of them and keeps those block-table
+ * entries (the pages stay mapped, unused), while its row_len is still set to new_len.
  */
 kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, const int32_t *move_dst,
                              const int32_t *num_moves, const int32_t *new_len, float *crf,
@@ -263,8 +274,7 @@ kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, co
 
 /*
  * kvc_compact_pages without a caller-provided workspace, for callers that cannot allocate
- * device memory: code running during CUDA graph capture (an allocation there breaks the
- * capture), engines whose allocator has given all free memory to the KV pool, or
+ * device memory: engines whose allocator has given all free memory to the KV pool, or
  * foreign-function callers with no access to the host framework's allocator.  The pages
  * describe no such variant; it exists for those callers only.
  * Same arguments, checks and results as kvc_compact_pages, minus workspace/workspace_bytes:

@@ -43,10 +43,28 @@ def geometry(spec: synth.Spec) -> ocache.Geometry:
     return ocache.Geometry(spec.num_seqs, spec.num_layers, spec.num_kv_heads, spec.num_q_heads, spec.page_size)
 
 
-def build(spec: synth.Spec, device="cuda") -> Workload:
+def randn_pool(spec: synth.Spec, layout: synth.Layout, seed: int, device="cuda") -> torch.Tensor:
+    """A pool of N(0, 1) values from torch's seeded generator, rounded to the spec dtype (fast at any size)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    pool = torch.empty((layout.num_pages, spec.page_size, spec.head_dim), dtype=synth.torch_dtype(spec), device=device)
+    flat = pool.view(-1)
+    step = 1 << 28
+    for a in range(0, flat.numel(), step):
+        b = min(flat.numel(), a + step)
+        flat[a:b] = torch.randn(b - a, generator=g, device=device, dtype=torch.float32).to(pool.dtype)
+    return pool
+
+
+def build(spec: synth.Spec, device="cuda", fill: str = "synth") -> Workload:
+    """Seeded workload on the device; fill="randn" draws the pools from torch's generator instead of the
+    counter-based one (for caches too large to generate element by element in reasonable time)."""
     layout = synth.make_layout(spec)
-    kp = synth.fill_pool(spec, layout, "k", device)
-    vp = synth.fill_pool(spec, layout, "v", device)
+    if fill == "randn":
+        kp = randn_pool(spec, layout, spec.seed * 2 + 1, device)
+        vp = randn_pool(spec, layout, spec.seed * 2 + 2, device)
+    else:
+        kp = synth.fill_pool(spec, layout, "k", device)
+        vp = synth.fill_pool(spec, layout, "v", device)
     qs = synth.make_queries(spec, device)
     lse = torch.full((spec.num_seqs, spec.num_layers, spec.num_q_heads, qs.max_q), float("-inf"),
                      dtype=torch.float32, device=device)

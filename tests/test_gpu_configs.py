@@ -4,9 +4,10 @@ compact) through ``EvictionRound``, beside the oracle run on the same seeded inp
 Chained rounds compare each step with the tolerance fixed for it: scores 1e-6 + 1e-3 relative;
 kept sets identical except entries whose oracle LRFU value lies within 1e-4 relative of the
 oracle's budget-th value, or whose score lies within 1e-4 relative of the oracle's gate threshold
-(the two places where fp32 against fp64 may legitimately flip a decision).  When the kept sets are
-identical the compacted state (pools, block table, positions, labels, row lengths, freed list) must
-equal the oracle's bit for bit.
+(the two places where fp32 against fp64 may legitimately flip a decision).  The oracle then plans and
+compacts with the GPU's keep mask, and the compacted state (pools, block table, positions, labels, row
+lengths, freed list) must equal the oracle's bit for bit; multi-round runs carry the oracle's state
+forward on the GPU's decisions wherever those sit in a tolerance band, so the two stay in lockstep.
 """
 import numpy as np
 import pytest
@@ -46,9 +47,29 @@ def snapshot(w):
                 rl=c.row_len.cpu().numpy(), sp=c.slot_pos.cpu().numpy(), sl=c.slot_label.cpu().numpy())
 
 
+def _orig_slots(src, dst, size):
+    """Slot j after compaction holds the entry that was at orig[j] before it."""
+    orig = np.arange(size)
+    orig[np.asarray(dst, dtype=np.int64)] = np.asarray(src, dtype=np.int64)
+    return orig
+
+
+def check_crf(gcrf, ocrf, osc, ohits, orig, m, what):
+    """CRF after compaction against the oracle's, entry by entry: within the score tolerance, except where the
+    GPU's hit decision sits in the gate-threshold band (then the two differ by that entry's hit)."""
+    want = ocrf[orig[:m]]
+    tau = osc[ohits].min() if ohits.any() else 0.0
+    band = np.abs(osc[orig[:m]] - tau) <= 1e-4 * tau
+    bad = np.abs(gcrf[:m] - want) > 1e-6 + 1e-3 * np.abs(want)
+    assert not (bad & ~band).any(), f"{what}: {int((bad & ~band).sum())} CRF values out of tolerance"
+    return bad & band
+
+
 def run_and_check(w, budgets, logits=None, rows=None):
-    """One chained round on the GPU and on the oracle (for `rows`, default all); returns True when the kept
-    sets were identical (then the compacted rows were also checked bit for bit)."""
+    """One chained round on the GPU and on the oracle (for `rows`, default all).  Scores and kept sets are compared
+    with their tolerances; then the oracle plans and compacts with the GPU's keep mask (identical to its own except
+    inside the tolerance bands), and the compacted rows, the freed list and (for whole-cache runs) every byte of
+    both pools must equal the GPU's bit for bit.  Returns the number of kept-set differences in the bands."""
     spec, geo, P = w.spec, w.geo, w.spec.page_size
     all_rows = rows is None
     rows = list(range(spec.rows)) if rows is None else rows
@@ -78,7 +99,9 @@ def run_and_check(w, budgets, logits=None, rows=None):
     osc = H.oracle_scores(w, lse32, rows, snaps)
     gsc = rnd.scores.cpu().numpy() if all_rows else {r: rnd.scores[r].cpu().numpy() for r in rows}
     gkeep = rnd.keep.cpu().numpy() if all_rows else {r: rnd.keep[r].cpu().numpy() for r in rows}
-    same, okeeps, ocrfs = True, {}, {}
+    gkept = rnd.kept.cpu().numpy()
+    gcrf_all = rnd.crf.cpu().numpy() if all_rows else {r: rnd.crf[r].cpu().numpy() for r in rows}
+    in_band = 0
     for r in rows:
         sn = snaps[r]
         n = sn.n
@@ -87,17 +110,21 @@ def run_and_check(w, budgets, logits=None, rows=None):
         ocrf = opath.lrfu_update(np.zeros(n), osc[r], sn.sp[:n], 0.5, HIT)
         ohit = opath.hit_gate(osc[r], sn.sp[:n], HIT)
         okeep = opath.select_budget(ocrf, sn.sp[:n], int(budgets[s]))
-        okeeps[r], ocrfs[r] = okeep, ocrf
-        same &= check_keep(gkeep[r][:n], okeep, ocrf, osc[r], ohit, int(budgets[s]))
-    if not same:
-        return False
-    # compaction of each checked row, on its own pages, against the device state
+        gk = gkeep[r][:n].astype(bool)
+        if not check_keep(gk, okeep, ocrf, osc[r], ohit, int(budgets[s])):
+            in_band += int((gk != okeep).sum())
+        assert int(gk.sum()) == min(int(budgets[s]), n) == int(gkept[r])
+        assert not gkeep[r][n:].any()
+        # CRF moved by the compaction: the GPU's LRFU value of each surviving entry
+        src, dst, m = opath.plan_slots(gk, n)
+        check_crf(gcrf_all[r], ocrf, osc[r], ohit, _orig_slots(src, dst, n), m, f"row {r}")
+    # compaction of each checked row on the GPU's keep mask, on its own pages, against the device state
     rl1 = w.cache.row_len.cpu().numpy()
     off = np.concatenate([[0], np.cumsum([-(-int(a) // P) - (-(-int(b) // P)) for a, b in zip(rl0, rl1)])])
     freed_dev = rnd.freed.cpu().numpy()
     for r in rows:
         sn = snaps[r]
-        src, dst, m = opath.plan_slots(okeeps[r], sn.n)
+        src, dst, m = opath.plan_slots(gkeep[r][:sn.n].astype(bool), sn.n)
         row = opath.PagedRow(block_table=np.arange(len(sn.pages)), n=sn.n, slot_pos=sn.sp.copy(),
                              slot_label=sn.sl.copy(), crf=None)
         k2, v2, new, freed_local = opath.compact_row(sn.kbits, sn.vbits, row, src, dst, m, P)
@@ -113,13 +140,13 @@ def run_and_check(w, budgets, logits=None, rows=None):
         assert np.array_equal(freed_dev[off[r]:off[r + 1]], sn.pages[freed_local])
     if all_rows:
         # the entire pool: pages of no row, and every byte of every row, as the oracle's gather compaction
-        plans = {r: opath.plan_slots(okeeps[r], snaps[r].n) for r in rows}
+        plans = {r: opath.plan_slots(gkeep[r][:snaps[r].n].astype(bool), snaps[r].n) for r in rows}
         k2, v2, *_ , fr = ocache.compact_cache(geo, full0["k"], full0["v"], full0["bt"], full0["rl"], full0["sp"],
                                                 full0["sl"], None, plans)
         st1 = snapshot(w)
         assert np.array_equal(st1["k"], k2) and np.array_equal(st1["v"], v2)
         assert int(rnd.num_freed[0]) == len(fr) and np.array_equal(freed_dev[:len(fr)], fr)
-    return True
+    return in_band
 
 
 @pytest.mark.parametrize("variant", [0, 1])
@@ -127,7 +154,7 @@ def test_tiny_round(variant):
     """1 seq, 4 q / 2 KV heads, D 64, fp32, 1,024 tokens in shuffled pages, 8 action queries, budget 256."""
     spec = synth.tiny(variant=variant)
     w = H.build(spec)
-    assert run_and_check(w, [spec.budget])
+    assert run_and_check(w, [spec.budget]) == 0
 
 
 @pytest.mark.parametrize("ctx", [4096 + 99, 32768])
@@ -137,7 +164,7 @@ def test_llama8b_layer_round(ctx):
     spec = synth.llama8b_layer(ctx=ctx)
     w = H.build(spec)
     logits = torch.stack([synth.logits(spec, 0, 0, 64, device=DEV)])
-    run_and_check(w, None, logits=logits)
+    assert run_and_check(w, None, logits=logits) <= 2
 
 
 def test_batch_round_small():
@@ -145,99 +172,179 @@ def test_batch_round_small():
     spec = synth.batch16(num_seqs=3, num_layers=2, lo=1500, hi=3500)
     w = H.build(spec)
     logits = torch.stack([synth.logits(spec, s, 0, 64, device=DEV) for s in range(spec.num_seqs)])
-    run_and_check(w, None, logits=logits)
+    assert run_and_check(w, None, logits=logits) <= 2 * spec.rows
 
 
 def test_batch16_full_sampled():
-    """Batch 16 x 32 layers x 8 KV heads at 8K-33K context (all rows scored on the GPU); the oracle checks
-    four sampled rows end to end."""
+    """Batch 16 x 32 layers x 8 KV heads at 8K-33K context (all rows scored on the GPU); the oracle checks 32
+    sampled rows end to end (every sequence at least once, the first and the last row among them)."""
     spec = synth.batch16()
     w = H.build(spec)
     logits = torch.stack([synth.logits(spec, s, 0, 64, device=DEV) for s in range(spec.num_seqs)])
-    rows = [0, spec.row_id(5, 17, 3), spec.row_id(11, 31, 7), spec.rows - 1]
-    run_and_check(w, None, logits=logits, rows=rows)
+    rng = np.random.default_rng(3)
+    rows = {0, spec.rows - 1}
+    rows |= {spec.row_id(s, int(rng.integers(spec.num_layers)), int(rng.integers(spec.num_kv_heads)))
+             for s in range(spec.num_seqs)}
+    while len(rows) < 32:
+        rows.add(int(rng.integers(spec.rows)))
+    assert run_and_check(w, None, logits=logits, rows=sorted(rows)) <= 2 * len(rows)
 
 
-def test_streaming_rounds():
-    """Streaming shape: beacon + recent queries (LSE computed by the library), 28 q / 4 KV heads, the LRFU state
-    carried across rounds, 64 decoded tokens appended between compactions.  The oracle keeps its own state from
-    the initial generated cache onward; the appended tokens go to pages no block table references (the same
-    pages on both sides)."""
-    spec = synth.streaming(num_seqs=2, ctx=2048)
-    spec.spare_frac = 0.7
-    spec.budget = 1800
+class RowState:
+    """The oracle's own copy of one row: its logical pages (raw bits, local page order), positions, labels, CRF."""
+
+    def __init__(self, kb, vb, sp, sl, n, max_slots):
+        self.kb, self.vb, self.sp, self.sl, self.n = kb, vb, sp.astype(np.int64), sl.copy(), n
+        self.crf = np.zeros(max_slots)
+
+
+def append_tokens(w, rnd, n_total, free, states, count=64):
+    """Append `count` decoded tokens to every row (pages taken from the free list in order when a row needs one),
+    on the device and in the oracle's sampled rows; the values come from the seeded generator on both sides."""
+    spec, geo, P, D = w.spec, w.geo, w.spec.page_size, w.spec.head_dim
+    c = w.cache
+    bt = c.block_table.cpu().numpy()
+    rl = c.row_len.cpu().numpy()
+    phys, kv, vv, rows_idx, slots_all, pos_all = [], [], [], [], [], []
+    for r in range(spec.rows):
+        s, l, h = geo.coords(r)
+        m = int(rl[r])
+        for p in range(m // P, (m + count - 1) // P + 1):
+            if bt[r, p] < 0:
+                bt[r, p] = free.pop(0)
+        slots = np.arange(m, m + count)
+        pos = torch.arange(n_total[s], n_total[s] + count, dtype=torch.int64)
+        phys.append(bt[r, slots // P].astype(np.int64) * P + slots % P)
+        k = synth.key_values(spec, s, l, h, pos.to(DEV), "k")
+        v = synth.key_values(spec, s, l, h, pos.to(DEV), "v")
+        kv.append(k)
+        vv.append(v)
+        rows_idx.append(np.full(count, r))
+        slots_all.append(slots)
+        pos_all.append(pos.numpy())
+        if r in states:
+            st = states[r]
+            need = (m + count + P - 1) // P
+            if st.kb.shape[0] < need:
+                extra = need - st.kb.shape[0]
+                st.kb = np.concatenate([st.kb, np.zeros((extra, P, D), dtype=st.kb.dtype)])
+                st.vb = np.concatenate([st.vb, np.zeros((extra, P, D), dtype=st.vb.dtype)])
+            st.kb.reshape(-1, D)[slots] = H._bits(k).cpu().numpy()
+            st.vb.reshape(-1, D)[slots] = H._bits(v).cpu().numpy()
+            st.sp[slots] = pos.numpy()
+            st.sl[slots] = synth.LABEL_REASON
+            st.crf[slots] = 0.0
+            st.n = m + count
+    ph = torch.from_numpy(np.concatenate(phys)).to(DEV)
+    c.k_pool.view(-1, D)[ph] = torch.cat(kv)
+    c.v_pool.view(-1, D)[ph] = torch.cat(vv)
+    ri = torch.from_numpy(np.concatenate(rows_idx)).to(DEV)
+    si = torch.from_numpy(np.concatenate(slots_all)).to(DEV)
+    c.slot_pos[ri, si] = torch.from_numpy(np.concatenate(pos_all).astype(np.int32)).to(DEV)
+    c.slot_label[ri, si] = synth.LABEL_REASON
+    rnd.crf[ri, si] = 0.0
+    c.block_table.copy_(torch.from_numpy(bt))
+    c.row_len.copy_(torch.from_numpy(rl + count))
+    for s in range(spec.num_seqs):
+        n_total[s] += count
+
+
+def streaming_lockstep(spec, rounds, sample):
+    """Streaming rounds in lockstep with the oracle on the sampled rows: beacon + recent queries with the LSE
+    computed by the library, the LRFU state carried across rounds, 64 decoded tokens appended after each
+    compaction.  Every round compares the LSE, scores, kept set, CRF and the compacted row (pages bit for bit,
+    positions, labels, freed pages); the oracle then carries on from the GPU's keep mask and, where a hit decision
+    sits in the gate-threshold band, from the GPU's CRF value, so that its state follows the GPU's."""
     w = H.build(spec)
-    geo, P, D = w.geo, spec.page_size, spec.head_dim
+    geo, P, G = w.geo, spec.page_size, spec.group
     rnd = EvictionRound(w.cache)
     rnd.budget.fill_(spec.budget)
-    o = snapshot(w)                      # oracle state: the generated cache, before any kernel ran
-    o["crf"] = np.zeros((spec.rows, spec.max_slots))
-    in_use = set(int(x) for x in o["bt"][o["bt"] >= 0])
+    snaps = H.snap_rows(w, sample)
+    states = {r: RowState(snaps[r].kbits, snaps[r].vbits, snaps[r].sp, snaps[r].sl, snaps[r].n, spec.max_slots)
+              for r in sample}
+    bt0 = w.cache.block_table.cpu().numpy()
+    in_use = set(int(x) for x in bt0[bt0 >= 0])
     free = [p for p in range(w.layout.num_pages) if p not in in_use]
-    n_total = [2048] * spec.num_seqs
-    for rd in range(10):
+    n_total = list(spec.ctx)
+    band_total = 0
+    for rd in range(rounds):
+        bt_before = w.cache.block_table.cpu().numpy()
+        rl_before = w.cache.row_len.cpu().numpy()
         qs = synth.streaming_queries(spec, n_total, device=DEV)
         q = kvc.QuerySet(qs.q, torch.zeros((spec.num_seqs, 1, spec.num_q_heads, qs.max_q), device=DEV),
                          qs.q_pos, qs.num_q)
         rnd.run(q, None, hit_mass=HIT, score_flags=kvc.KVC_SCORE_COMPUTE_LSE)
         torch.cuda.synchronize()
-        assert rnd.device_status()[0] == 0
-        hq = qs.q.cpu().to(torch.float64).numpy()
-        qpos, numq = qs.q_pos.cpu().numpy(), qs.num_q.cpu().numpy()
-        kf = torch.from_numpy(o["k"]).view(torch.bfloat16).to(torch.float64).numpy()
-        lse_o = ocache.lse_cache(geo, kf, o["bt"], o["rl"], o["sp"], hq, qpos, numq, qs.max_q)
-        glse = q.lse.cpu().numpy().astype(np.float64)
-        assert np.max(np.abs(glse - lse_o)) < 5e-5, "the library's LSE pass against the oracle's"
-        osc = ocache.score_cache(geo, kf, o["bt"], o["rl"], o["sp"], hq, lse_o.astype(np.float32), qpos, numq)
-        crf_o, ohits = ocache.lrfu_cache(geo, osc, o["crf"], o["rl"], o["sp"], 0.5, HIT)
-        okeep, _ = ocache.select_cache(geo, crf_o, o["rl"], o["sp"], o["sl"], [spec.budget] * spec.num_seqs)
-        gsc, gkeep = rnd.scores.cpu().numpy(), rnd.keep.cpu().numpy()
-        same = True
-        for r in range(spec.rows):
-            n = int(o["rl"][r])
-            H.assert_scores_close(gsc[r, :n], osc[r, :n], f"round {rd} row {r}")
-            same &= check_keep(gkeep[r, :n], okeep[r, :n], crf_o[r, :n], osc[r, :n], ohits[r, :n], spec.budget)
-        if not same:
-            return   # both sides are right; their states part here
-        plans = ocache.plan_cache(geo, okeep, o["rl"])
-        k2, v2, bt2, rl2, sp2, sl2, crf2, fr = ocache.compact_cache(geo, o["k"], o["v"], o["bt"], o["rl"], o["sp"],
-                                                                    o["sl"], crf_o, plans)
-        st1 = snapshot(w)
-        for key, val in (("k", k2), ("v", v2), ("bt", bt2), ("rl", rl2), ("sp", sp2), ("sl", sl2)):
-            assert np.array_equal(st1[key], val), f"round {rd}: {key}"
-        gcrf = rnd.crf.cpu().numpy()
-        for r in range(spec.rows):
-            m = int(rl2[r])
-            np.testing.assert_allclose(gcrf[r, :m], crf2[r, :m], rtol=2e-5, atol=1e-30)
-        assert int(rnd.num_freed[0]) == len(fr)
-        free.extend(int(x) for x in fr)
-        # append 64 decoded tokens per row, to both states
-        o = dict(k=k2, v=v2, bt=bt2, rl=rl2, sp=sp2, sl=sl2, crf=crf2)
-        for r in range(spec.rows):
+        assert rnd.device_status()[0] == 0, (rd, rnd.device_status())
+        rl_after = w.cache.row_len.cpu().numpy()
+        bt_after = w.cache.block_table.cpu().numpy()
+        per_row = [-(-int(a) // P) - (-(-int(b) // P)) for a, b in zip(rl_before, rl_after)]
+        off = np.concatenate([[0], np.cumsum(per_row)])
+        nf = int(rnd.num_freed[0])
+        assert nf == off[-1]
+        freed_dev = rnd.freed[:nf].cpu().numpy()
+        qpos = qs.q_pos.cpu().numpy()
+        for r in sample:
+            st = states[r]
             s, l, h = geo.coords(r)
-            m = int(o["rl"][r])
-            pos = torch.arange(n_total[s], n_total[s] + 64)
-            for slot in range(m, m + 64):
-                if o["bt"][r, slot // P] < 0:
-                    o["bt"][r, slot // P] = free.pop(0)
-            slots = np.arange(m, m + 64)
-            phys = o["bt"][r, slots // P].astype(np.int64) * P + slots % P
-            kv = synth.key_values(spec, s, l, h, pos, "k")
-            vv = synth.key_values(spec, s, l, h, pos, "v")
-            o["k"].reshape(-1, D)[phys] = kv.view(torch.int16).numpy()
-            o["v"].reshape(-1, D)[phys] = vv.view(torch.int16).numpy()
-            w.cache.k_pool.view(-1, D)[torch.from_numpy(phys).to(DEV)] = kv.to(DEV)
-            w.cache.v_pool.view(-1, D)[torch.from_numpy(phys).to(DEV)] = vv.to(DEV)
-            o["sp"][r, m:m + 64] = pos.numpy()
-            o["sl"][r, m:m + 64] = synth.LABEL_REASON
-            o["rl"][r] = m + 64
-            o["crf"][r, m:m + 64] = 0.0
-            rnd.crf[r, m:m + 64] = 0.0
-        w.cache.block_table.copy_(torch.from_numpy(o["bt"]))
-        w.cache.row_len.copy_(torch.from_numpy(o["rl"]))
-        w.cache.slot_pos.copy_(torch.from_numpy(o["sp"]))
-        w.cache.slot_label.copy_(torch.from_numpy(o["sl"]))
-        n_total = [n + 64 for n in n_total]
+            n = st.n
+            assert int(rl_before[r]) == n
+            what = f"round {rd} row {r}"
+            kf = torch.from_numpy(st.kb.reshape(-1, spec.head_dim)[:n]).view(torch.bfloat16).to(torch.float64).numpy()
+            qg = qs.q[s, l, :, h * G:(h + 1) * G].cpu().to(torch.float64).numpy()
+            lse_o = opath.attention_lse(qg, kf, qpos[s], st.sp[:n])
+            glse = q.lse[s, l, h * G:(h + 1) * G].cpu().numpy().astype(np.float64)
+            assert np.max(np.abs(glse - lse_o)) < 5e-5, f"{what}: the library's LSE pass against the oracle's"
+            osc = opath.scores_from_lse(qg, kf, qpos[s], st.sp[:n], lse_o.astype(np.float32).astype(np.float64))
+            H.assert_scores_close(rnd.scores[r, :n].cpu().numpy(), osc, what)
+            ohit = opath.hit_gate(osc, st.sp[:n], HIT)
+            ocrf = opath.lrfu_update(st.crf[:n], osc, st.sp[:n], 0.5, HIT)
+            okeep = opath.select_budget(ocrf, st.sp[:n], spec.budget)
+            gk = rnd.keep[r, :n].cpu().numpy().astype(bool)
+            if not check_keep(gk, okeep, ocrf, osc, ohit, spec.budget):
+                band_total += int((gk != okeep).sum())
+            # the oracle compacts on the GPU's keep mask
+            src, dst, m = opath.plan_slots(gk, n)
+            crf_full = st.crf.copy()
+            crf_full[:n] = ocrf
+            npg = -(-n // P)
+            row = opath.PagedRow(block_table=np.arange(npg), n=n, slot_pos=st.sp.copy(), slot_label=st.sl.copy(),
+                                 crf=crf_full)
+            kb2, vb2, new, freed_local = opath.compact_row(st.kb[:npg], st.vb[:npg], row, src, dst, m, P)
+            kp = -(-m // P)
+            assert int(rl_after[r]) == m, what
+            assert np.array_equal(bt_after[r, :kp], bt_before[r, :kp]) and np.all(bt_after[r, kp:npg] == -1), what
+            pg = torch.from_numpy(bt_after[r, :kp].astype(np.int64)).to(DEV)
+            assert np.array_equal(H._bits(w.cache.k_pool[pg]).cpu().numpy(), kb2[:kp]), what
+            assert np.array_equal(H._bits(w.cache.v_pool[pg]).cpu().numpy(), vb2[:kp]), what
+            assert np.array_equal(w.cache.slot_pos[r].cpu().numpy(), new.slot_pos.astype(np.int32)), what
+            assert np.array_equal(w.cache.slot_label[r].cpu().numpy(), new.slot_label), what
+            assert np.array_equal(freed_dev[off[r]:off[r + 1]], bt_before[r, freed_local]), what
+            gcrf = rnd.crf[r].cpu().numpy().astype(np.float64)
+            adopt = check_crf(gcrf, ocrf, osc, ohit, _orig_slots(src, dst, n), m, what)
+            new.crf[:m][adopt] = gcrf[:m][adopt]
+            st.kb, st.vb, st.sp, st.sl, st.crf, st.n = kb2[:kp], vb2[:kp], new.slot_pos, new.slot_label, new.crf, m
+        free.extend(int(x) for x in freed_dev)
+        if rd + 1 < rounds:
+            append_tokens(w, rnd, n_total, free, states)
+    return band_total
+
+
+def test_streaming_rounds():
+    """Streaming shape scaled down: 2 sequences x 2,048 tokens, 28 q / 4 KV heads, budget 1,800, 30 rounds, every
+    row checked in lockstep."""
+    spec = synth.streaming(num_seqs=2, ctx=2048)
+    spec.spare_frac = 0.05
+    spec.budget = 1800
+    assert streaming_lockstep(spec, 30, list(range(spec.rows))) <= 30 * spec.rows
+
+
+def test_streaming_rounds_full():
+    """The streaming workload at size: 8 sequences x 32K tokens growing by 64 decoded tokens per round, 28 q / 4 KV
+    heads, budget 30,000, 200 rounds; four sampled rows checked in lockstep every round."""
+    spec = synth.streaming()
+    sample = [0, spec.row_id(3, 0, 1), spec.row_id(5, 0, 2), spec.rows - 1]
+    assert streaming_lockstep(spec, 200, sample) <= 200 * len(sample)
 
 
 def _stress_cache(S, L, ctx, seed, device=DEV):
@@ -255,6 +362,23 @@ def _stress_cache(S, L, ctx, seed, device=DEV):
     cache = kvc.Cache(pools[0], pools[1], layout.block_table.to(device), layout.row_len.to(device),
                       layout.slot_pos.to(device), layout.slot_label.to(device), S, L, spec.num_kv_heads)
     return spec, layout, cache
+
+
+def test_stress_scored_round_sampled():
+    """The stress shape through a whole scored round: 64 sequences x 33,000 tokens (partial last page) x 4 layers x
+    8 KV heads, 32 q heads, action-token queries, a budget that frees 40% of every row's pages; all 2,048 rows are
+    scored, gated, selected, planned and compacted on the GPU and eight sampled rows are checked end to end."""
+    spec = synth.stress(num_seqs=64, num_layers=4, ctx=33000)
+    spec.queries = "action"
+    w = H.build(spec, fill="randn")
+    B = synth.stress_budget(spec.ctx[0])
+    rng = np.random.default_rng(8)
+    rows = sorted({0, spec.rows - 1} | {int(x) for x in rng.choice(spec.rows, size=6, replace=False)})
+    assert run_and_check(w, [B] * spec.num_seqs, rows=rows) <= 2 * len(rows)
+    pages = -(-spec.ctx[0] // spec.page_size)
+    assert pages - (-(-B // spec.page_size)) == int(round(0.4 * pages))
+    del w
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("size", ["small", "full"])

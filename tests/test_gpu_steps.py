@@ -354,6 +354,44 @@ def test_compact_freed_overflow_keeps_pages():
     assert c.row_len.cpu().tolist() == [16, 16]
 
 
+def test_plan_mismatch_leaves_row_untouched():
+    """A row whose kept count disagrees with its keep mask is reported (kept mismatch), gets num_moves = -1 and is
+    left exactly as it was by the compaction: block table, row_len, positions and pool bytes; the consistent row
+    beside it is compacted as usual."""
+    lengths = [64, 64]
+    c = bare_cache(lengths, 64, S=2)
+    keep = np.zeros((2, 64), dtype=np.uint8)
+    keep[0, 40:56] = 1
+    keep[1, 30:50] = 1
+    kept = np.array([16, 16], dtype=np.int32)          # row 1's mask holds 20 entries
+    src = torch.zeros((2, 64), dtype=torch.int32, device=DEV)
+    dst = torch.zeros((2, 64), dtype=torch.int32, device=DEV)
+    nm = torch.zeros(2, dtype=torch.int32, device=DEV)
+    status = torch.zeros(2, dtype=torch.int32, device=DEV)
+    kd = torch.from_numpy(kept).to(DEV)
+    bt0, rl0, sp0 = c.block_table.cpu().numpy().copy(), c.row_len.cpu().numpy().copy(), c.slot_pos.cpu().numpy().copy()
+    k0 = c.k_pool.cpu().view(torch.int16).numpy().copy()
+    v0 = c.v_pool.cpu().view(torch.int16).numpy().copy()
+    kvc.kvc_plan_slots(c, torch.from_numpy(keep).to(DEV), kd, src, dst, nm, status)
+    freed = torch.full((16,), -1, dtype=torch.int32, device=DEV)
+    nfreed = torch.zeros(1, dtype=torch.int64, device=DEV)
+    ws = torch.zeros(8, dtype=torch.int64, device=DEV)
+    kvc.kvc_compact_pages(c, src, dst, nm, kd, None, freed, nfreed, ws, status)
+    torch.cuda.synchronize()
+    assert kvc.device_status(status)[:2] == (4, 1)
+    assert nm.cpu().tolist() == [16, -1]
+    bt1 = c.block_table.cpu().numpy()
+    assert np.array_equal(bt1[1], bt0[1]) and int(c.row_len[1]) == 64
+    assert np.array_equal(c.slot_pos.cpu().numpy()[1], sp0[1])
+    pages1 = bt0[1, :4].astype(np.int64)
+    assert np.array_equal(c.k_pool.cpu().view(torch.int16).numpy()[pages1], k0[pages1])
+    assert np.array_equal(c.v_pool.cpu().view(torch.int16).numpy()[pages1], v0[pages1])
+    # row 0: 16 survivors moved into the first page, three pages freed
+    assert int(c.row_len[0]) == 16 and int(nfreed[0]) == 3
+    assert freed.cpu().tolist()[:3] == bt0[0, 1:4].tolist()
+    assert np.array_equal(c.slot_pos.cpu().numpy()[0, :16], sp0[0, 40:56])
+
+
 # ----------------------------------------------------------------------------- confidence + ratchet
 
 @pytest.mark.parametrize("V", [4096 + 13, 128256])

@@ -32,6 +32,14 @@ def test_library_exports_every_declared_entry_point():
     assert set(kvc.EXPORTS) == set(names)
 
 
+def test_noalloc_row_limit_matches_header():
+    """The binding's copy of KVC_NOALLOC_MAX_ROWS is the header's value (the GPU test builds its over-limit case
+    from the binding's copy)."""
+    with open(os.path.join(ROOT, "include", "kvc.h")) as f:
+        m = re.search(r"#define\s+KVC_NOALLOC_MAX_ROWS\s+(\d+)", f.read())
+    assert m and int(m.group(1)) == kvc.NOALLOC_MAX_ROWS
+
+
 def test_struct_layouts_match_header_sizes():
     # kvc_cache: 2 pointers + int64 + 4 int32 + 4 pointers + 4 int32 (with padding) on LP64
     assert ctypes.sizeof(kvc.KvcCache) == 2 * 8 + 8 + 4 * 4 + 4 * 8 + 4 * 4

@@ -1,8 +1,8 @@
 """The compaction entry point that allocates nothing, against the regular one.
 
-Some callers cannot allocate device memory when they compact: code that runs while a CUDA
-graph is being captured, engines whose allocator has handed all free memory to the KV pool,
-or foreign-function callers with no access to the host framework's allocator.  For them
+Some callers cannot allocate device memory when they compact: engines whose allocator has
+handed all free memory to the KV pool, or foreign-function callers with no access to the host
+framework's allocator.  For them
 kvc_compact_pages_noalloc keeps its workspace in an array inside the library.  This test
 calls both entry points through the C ABI on identical copies of a cache and requires the
 same results (compaction is bit-exact), on two calls in a row so that whatever the first
