@@ -54,7 +54,7 @@ def check_fp32(c32: np.ndarray, n: int = 2_000_001):
 
 
 if __name__ == "__main__":
-    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 4
+    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 5
     c, e = remez_relative(deg)
     c32 = c.astype(np.float32)
     print(f"degree {deg}: minimax relative error {e:.3e}; fp32 Horner {check_fp32(c32):.3e}")

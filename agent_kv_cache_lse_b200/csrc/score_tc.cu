@@ -246,20 +246,24 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // 2^x on the FMA pipes for a pair of arguments: x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a
-// degree-3 polynomial whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
-// exchange, derived by exp2_poly.py beside this file: max relative error 7.5e-5); 2^n enters through the
-// exponent bits.  x is clamped at -126 so the exponent arithmetic stays in range (the result is then
-// ~1e-38).  The floating-point steps run as packed f32x2 operations.
+// degree-5 polynomial whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange, derived by exp2_poly.py beside this file: 2.4e-7 relative in fp32 Horner form, the accuracy
+// class of the MUFU unit's approximation, so that the two kinds of exponential are interchangeable under a
+// 1e-4 ranking tolerance); 2^n enters through the exponent bits.  x is clamped at -126 so the exponent
+// arithmetic stays in range (the result is then ~1e-38).  The floating-point steps run as packed f32x2
+// operations.
 __device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
-                    kC3 = 0.0551716685295105f;
+    constexpr float kC0 = 1.0000001192092896f, kC1 = 0.6931469440460205f, kC2 = 0.24022120237350464f,
+                    kC3 = 0.05550713092088699f, kC4 = 0.009675540961325169f, kC5 = 0.0013276472454890609f;
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
     x.x = fmaxf(x.x, -126.0f);
     x.y = fmaxf(x.y, -126.0f);
     const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
     const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
     const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-    float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    float2 p = __ffma2_rn(make_float2(kC5, kC5), f, make_float2(kC4, kC4));
+    p = __ffma2_rn(p, f, make_float2(kC3, kC3));
+    p = __ffma2_rn(p, f, make_float2(kC2, kC2));
     p = __ffma2_rn(p, f, make_float2(kC1, kC1));
     p = __ffma2_rn(p, f, make_float2(kC0, kC0));
     return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),

@@ -63,9 +63,16 @@ class EvictionRound:
 
         With logits, the ratchet runs on a second stream beside the LRFU update (neither needs the other;
         the selection needs both), forked after the scores and joined before the selection."""
+        main = stream if stream is not None else torch.cuda.current_stream()
+        kvc.kvc_score_from_lse(self.cache, queries, self.scores, score_flags, self.status, main)
+        self.run_after_scores(logits, lam, hit_mass, main, protect_label_mask, confidence_out)
+
+    def run_after_scores(self, logits: Optional[torch.Tensor], lam: float = 0.5, hit_mass: float = 0.9, stream=None,
+                         protect_label_mask: int = 0, confidence_out: Optional[torch.Tensor] = None):
+        """Enqueue the rest of a round on scores already in self.scores: (ratchet | LRFU) -> select -> plan ->
+        compact, or LRFU + select in one launch when there are no logits."""
         c = self.cache
         main = stream if stream is not None else torch.cuda.current_stream()
-        kvc.kvc_score_from_lse(c, queries, self.scores, score_flags, self.status, main)
         if logits is not None:
             # the LRFU update goes first so that its clusters take their SMs before the ratchet's CTAs spread
             self._fork.record(main)

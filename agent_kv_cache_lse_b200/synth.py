@@ -347,17 +347,23 @@ def make_queries(spec: Spec, device="cpu") -> Queries:
     q = torch.zeros((S, L, max_q, Hq, D), dtype=torch_dtype(spec), device=device)
     q_pos = torch.full((S, max_q), -1, dtype=torch.int32)
     num_q = torch.zeros(S, dtype=torch.int32)
-    j = torch.arange(max_q, device=device, dtype=torch.int64)
-    hh = torch.arange(Hq, device=device, dtype=torch.int64)
-    d = torch.arange(D, device=device, dtype=torch.int64)
     for s in range(S):
         nq = len(pos_list[s])
         q_pos[s, :nq] = pos_list[s]
         num_q[s] = nq
         for l in range(L):
-            c = counter(s, l, hh[None, :, None], j[:nq, None, None], d[None, None, :])
-            q[s, l, :nq] = normal(spec.seed, S_Q, c).to(torch_dtype(spec))
+            q[s, l, :nq] = query_vectors(spec, s, l, nq, device)
     return Queries(q=q, q_pos=q_pos.to(device), num_q=num_q.to(device), max_q=max_q)
+
+
+def query_vectors(spec: Spec, s: int, l: int, nq: int, device="cpu") -> torch.Tensor:
+    """Query vectors [nq, Hq, D] of sequence s, layer l (action/fixed query sets: the query index is the
+    counter field), in the spec dtype; what make_queries places at q[s, l, :nq]."""
+    j = torch.arange(nq, device=device, dtype=torch.int64)
+    hh = torch.arange(spec.num_q_heads, device=device, dtype=torch.int64)
+    d = torch.arange(spec.head_dim, device=device, dtype=torch.int64)
+    c = counter(s, l, hh[None, :, None], j[:, None, None], d[None, None, :])
+    return normal(spec.seed, S_Q, c).to(torch_dtype(spec))
 
 
 def logits(spec: Spec, s: int, step0: int, steps: int, device="cpu") -> torch.Tensor:
