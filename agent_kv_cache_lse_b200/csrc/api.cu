@@ -135,6 +135,8 @@ kvc_status kvc_query_lse(const kvc_cache *cache, const kvc_queries *queries, int
     kvc_status s = view_cache(cache, c, true);
     if (s != KVC_OK) return s;
     if ((s = view_queries(queries, c, q)) != KVC_OK) return s;
+    if (kvc::lse_tc_supported(c, q))
+        return cuda_status(kvc::launch_lse_tc(c, q, d_status, (cudaStream_t)stream), "kvc_query_lse launch");
     return cuda_status(kvc::launch_lse_simt(c, q, d_status, (cudaStream_t)stream), "kvc_query_lse launch");
 }
 
@@ -151,13 +153,18 @@ kvc_status kvc_score_from_lse(const kvc_cache *cache, const kvc_queries *queries
         return fail(KVC_ERR_INVALID_ARGUMENT, "unknown flags");
     cudaStream_t st = (cudaStream_t)stream;
     if (flags & KVC_SCORE_COMPUTE_LSE) {
-        if ((s = cuda_status(kvc::launch_lse_simt(c, q, d_status, st), "lse launch")) != KVC_OK) return s;
+        const bool tc = kvc::lse_tc_supported(c, q) && !(flags & KVC_SCORE_SIMT);
+        if ((s = cuda_status(tc ? kvc::launch_lse_tc(c, q, d_status, st) : kvc::launch_lse_simt(c, q, d_status, st),
+                             "lse launch")) != KVC_OK)
+            return s;
     }
     const bool acc = (flags & KVC_SCORE_ACCUMULATE) != 0;
     if (c.dtype == KVC_BF16 && !(flags & KVC_SCORE_SIMT)) {
         if (c.page_size != 16) return fail(KVC_ERR_UNSUPPORTED, "tensor-core scoring needs page_size 16");
         char err[256] = "";
-        cudaError_t e = kvc::launch_score_tc(c, q, scores, acc, d_status, st, err, sizeof(err));
+        cudaError_t e = kvc::score_pair_supported(c, q)
+                            ? kvc::launch_score_pair(c, q, scores, acc, d_status, st, err, sizeof(err))
+                            : kvc::launch_score_tc(c, q, scores, acc, d_status, st, err, sizeof(err));
         if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "score (tensor cores): %s %s", cudaGetErrorString(e), err);
         return KVC_OK;
     }
@@ -249,6 +256,32 @@ kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, co
                                            num_freed, static_cast<int64_t *>(workspace), d_status,
                                            (cudaStream_t)stream),
                        "kvc_compact_pages launch");
+}
+
+size_t kvc_append_workspace_bytes(int32_t rows) {
+    return rows < 0 ? 0 : (2 * (size_t)rows + 2) * sizeof(int64_t);
+}
+
+kvc_status kvc_append_tokens(const kvc_cache *cache, const void *k_new, const void *v_new, const int32_t *new_pos,
+                             int32_t count, uint8_t label, float *crf, int32_t *free_pages, int64_t *free_count,
+                             void *workspace, size_t workspace_bytes, int32_t *d_status, kvc_stream_t stream) {
+    g_err[0] = 0;
+    kvc::CacheView c;
+    kvc_status s = view_cache(cache, c, true);
+    if (s != KVC_OK) return s;
+    if (count < 0) return fail(KVC_ERR_INVALID_ARGUMENT, "count must be >= 0");
+    if (count == 0) return KVC_OK;
+    if (!k_new || !v_new || !new_pos || !free_pages || !free_count)
+        return fail(KVC_ERR_INVALID_ARGUMENT, "k_new, v_new, new_pos, free_pages and free_count are required");
+    const int esize = c.dtype == KVC_BF16 ? 2 : 4;
+    if ((c.head_dim * esize) % 16) return fail(KVC_ERR_UNSUPPORTED, "head_dim * element size must be a multiple of 16");
+    if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return fail(KVC_ERR_INVALID_ARGUMENT, "k_new and v_new must be 16-byte aligned");
+    if (!workspace || workspace_bytes < kvc_append_workspace_bytes(c.rows) || ((uintptr_t)workspace & 7))
+        return fail(KVC_ERR_INVALID_ARGUMENT, "workspace must be 8-byte aligned and at least %zu bytes",
+                    kvc_append_workspace_bytes(c.rows));
+    return cuda_status(kvc::launch_append(c, k_new, v_new, new_pos, count, label, crf, free_pages, free_count,
+                                          static_cast<int64_t *>(workspace), d_status, (cudaStream_t)stream),
+                       "kvc_append_tokens launch");
 }
 
 size_t kvc_ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params *params) {

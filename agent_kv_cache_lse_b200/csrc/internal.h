@@ -37,6 +37,13 @@ cudaError_t launch_score_simt(const CacheView &c, const QueryView &q, float *sco
 cudaError_t launch_lse_simt(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream);
 cudaError_t launch_score_tc(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
                             int32_t *status, cudaStream_t stream, char *err, size_t errlen);
+// Pair-of-SMs tensor-core scoring (bf16, head_dim 64 or 128, group size <= 128, query set within 256 blocks).
+bool score_pair_supported(const CacheView &c, const QueryView &q);
+cudaError_t launch_score_pair(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
+                              int32_t *status, cudaStream_t stream, char *err, size_t errlen);
+// Tensor-core LSE pass (bf16, head_dim 64 or 128, group size <= 128).
+bool lse_tc_supported(const CacheView &c, const QueryView &q);
+cudaError_t launch_lse_tc(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream);
 cudaError_t launch_lrfu(const CacheView &c, const float *scores, float *crf, float decay, float hit_mass,
                         bool binary, int32_t *status, cudaStream_t stream);
 cudaError_t launch_select(const CacheView &c, const float *crf, const int32_t *budget, uint32_t protect,
@@ -50,6 +57,9 @@ cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const in
                            const int32_t *num_moves, const int32_t *new_len, float *crf, int32_t *freed,
                            int64_t freed_capacity, int64_t *num_freed, int64_t *row_offsets,
                            int32_t *status, cudaStream_t stream);
+cudaError_t launch_append(const CacheView &c, const void *k_new, const void *v_new, const int32_t *new_pos,
+                          int32_t count, uint8_t label, float *crf, int32_t *free_pages, int64_t *free_count,
+                          int64_t *ws, int32_t *status, cudaStream_t stream);
 cudaError_t launch_beacon(const void *q, const int32_t *num_q, int32_t num_seqs, int32_t num_layers,
                           int32_t num_q_heads, int32_t head_dim, int32_t max_q, bool bf16, float *beacons,
                           int32_t *counts, int32_t num_beacons, void *beacon_q, int32_t out_max_q, int32_t *status,

@@ -29,7 +29,7 @@ EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse"
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
            "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select", "kvc_decode_attention",
-           "kvc_step_scores"]
+           "kvc_step_scores", "kvc_append_workspace_bytes", "kvc_append_tokens"]
 
 
 class KvcCache(ctypes.Structure):
@@ -102,6 +102,9 @@ def lib() -> ctypes.CDLL:
                                                  vp, vp]),
             "kvc_decode_attention": (ctypes.c_int, [pc, vp, vp, i32, vp, vp, vp, u32, vp, vp]),
             "kvc_step_scores": (ctypes.c_int, [pc, vp, vp, vp, i32, f32, vp, vp, vp]),
+            "kvc_append_workspace_bytes": (ctypes.c_size_t, [i32]),
+            "kvc_append_tokens": (ctypes.c_int, [pc, vp, vp, vp, i32, ctypes.c_uint8, vp, vp, vp, vp, ctypes.c_size_t,
+                                                 vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -255,6 +258,27 @@ def kvc_compact_pages_noalloc(cache: Cache, move_src, move_dst, num_moves, new_l
 
 
 NOALLOC_MAX_ROWS = 16384
+
+
+def kvc_append_workspace_bytes(rows: int) -> int:
+    return int(lib().kvc_append_workspace_bytes(rows))
+
+
+def kvc_append_tokens(cache: Cache, k_new: torch.Tensor, v_new: torch.Tensor, new_pos: torch.Tensor, label: int,
+                      crf: Optional[torch.Tensor], free_pages: torch.Tensor, free_count: torch.Tensor,
+                      workspace: torch.Tensor, d_status=None, stream=None):
+    """Append k_new/v_new [rows][count][D] at each row's end, pages from the free_pages stack (depth free_count)."""
+    count = k_new.shape[1]
+    _expect(k_new, "k_new", (cache.rows, count, cache.k_pool.shape[-1]), cache.k_pool.dtype)
+    _expect(v_new, "v_new", (cache.rows, count, cache.k_pool.shape[-1]), cache.k_pool.dtype)
+    _expect(new_pos, "new_pos", (cache.num_seqs, count), torch.int32)
+    if crf is not None:
+        _expect(crf, "crf", (cache.rows, cache.max_slots), torch.float32)
+    cs = cache.struct()
+    _check(lib().kvc_append_tokens(ctypes.byref(cs), _ptr(k_new), _ptr(v_new), _ptr(new_pos), count, label, _ptr(crf),
+                                   _ptr(free_pages), _ptr(free_count), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _ptr(d_status), _stream(stream)),
+           "kvc_append_tokens")
 
 
 def kvc_ratchet_state_bytes(num_seqs: int, params: KvcRatchetParams) -> int:

@@ -290,6 +290,28 @@ kvc_status kvc_compact_pages_noalloc(const kvc_cache *cache, const int32_t *move
                                      int32_t *freed, int64_t freed_capacity, int64_t *num_freed,
                                      int32_t *d_status, kvc_stream_t stream);
 
+/* bytes of device workspace kvc_append_tokens needs for `rows` rows */
+size_t kvc_append_workspace_bytes(int32_t rows);
+
+/*
+ * Streaming a compacted cache forward ("KV-streams for Efficient Compaction in Agentic Reinforcement
+ * Learning", abstract: the compacted cache is carried across rollouts instead of flushed and prefilled
+ * again).  Appends `count` new tokens to every row: the K and V vectors of token i go to slot
+ * row_len + i (i < count); where a row reaches a logical page it does not hold, it takes a page from the
+ * top of the free-page stack (rows in order, each row's new pages in ascending logical order: row r's k-th
+ * new page is free_pages[depth - total + offset_r + k], offset_r the pages all lower rows take, total the
+ * pages of the call) and enters it in its block table; slot_pos = new_pos of the row's sequence,
+ * slot_label = label, crf (when not NULL) = 0 for the new slots; row_len += count; *free_count -= total.
+ * k_new, v_new: [rows][count][head_dim] in the cache dtype, 16-byte aligned; new_pos: [num_seqs][count]
+ * int32; free_pages: the stack (e.g. kvc_compact_pages' freed list), *free_count (device int64, in/out) its
+ * depth; workspace: kvc_append_workspace_bytes(rows) bytes of device memory.
+ * Device faults: a stack too shallow for the call appends nothing and reports KVC_DEV_FREED_OVERFLOW
+ * (row -1); a row that would exceed max_slots, or whose row_len is negative, is left alone and reported.
+ */
+kvc_status kvc_append_tokens(const kvc_cache *cache, const void *k_new, const void *v_new, const int32_t *new_pos,
+                             int32_t count, uint8_t label, float *crf, int32_t *free_pages, int64_t *free_count,
+                             void *workspace, size_t workspace_bytes, int32_t *d_status, kvc_stream_t stream);
+
 /* bytes of the ratchet state buffer for num_seqs sequences */
 size_t kvc_ratchet_state_bytes(int32_t num_seqs, const kvc_ratchet_params *params);
 

@@ -4,4 +4,4 @@ TEST INFRASTRUCTURE ONLY: imported by the test suite, the package smoke check an
 the CPU-baseline leg of the benchmark, never by the product path.  It shares no
 code with the CUDA library.
 """
-from . import path, cache, beacon, decode, stepkv  # noqa: F401
+from . import path, cache, beacon, decode, stepkv, stream  # noqa: F401

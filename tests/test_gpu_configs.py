@@ -198,53 +198,57 @@ class RowState:
         self.crf = np.zeros(max_slots)
 
 
-def append_tokens(w, rnd, n_total, free, states, count=64):
-    """Append `count` decoded tokens to every row (pages taken from the free list in order when a row needs one),
-    on the device and in the oracle's sampled rows; the values come from the seeded generator on both sides."""
+class FreeStack:
+    """The free pages as a device stack (the library's append takes pages from its top; compaction's freed pages
+    are pushed on it)."""
+
+    def __init__(self, pages, capacity):
+        self.pages = torch.full((capacity,), -1, dtype=torch.int32, device=DEV)
+        self.pages[:len(pages)] = torch.tensor(pages, dtype=torch.int32, device=DEV)
+        self.depth = torch.tensor([len(pages)], dtype=torch.int64, device=DEV)
+
+    def push(self, freed, n):
+        d = int(self.depth[0])
+        self.pages[d:d + n] = freed[:n]
+        self.depth += n
+
+
+def append_tokens(w, rnd, n_total, stack, states, count=64):
+    """Append `count` decoded tokens to every row through kvc_append_tokens (pages from the free stack), and the
+    same tokens to the oracle's sampled rows; the values come from the seeded generator on both sides."""
     spec, geo, P, D = w.spec, w.geo, w.spec.page_size, w.spec.head_dim
     c = w.cache
-    bt = c.block_table.cpu().numpy()
     rl = c.row_len.cpu().numpy()
-    phys, kv, vv, rows_idx, slots_all, pos_all = [], [], [], [], [], []
+    kv = torch.empty((spec.rows, count, D), dtype=c.k_pool.dtype, device=DEV)
+    vv = torch.empty_like(kv)
+    new_pos = torch.empty((spec.num_seqs, count), dtype=torch.int32, device=DEV)
+    for s in range(spec.num_seqs):
+        new_pos[s] = torch.arange(n_total[s], n_total[s] + count, dtype=torch.int32, device=DEV)
     for r in range(spec.rows):
         s, l, h = geo.coords(r)
-        m = int(rl[r])
-        for p in range(m // P, (m + count - 1) // P + 1):
-            if bt[r, p] < 0:
-                bt[r, p] = free.pop(0)
-        slots = np.arange(m, m + count)
-        pos = torch.arange(n_total[s], n_total[s] + count, dtype=torch.int64)
-        phys.append(bt[r, slots // P].astype(np.int64) * P + slots % P)
-        k = synth.key_values(spec, s, l, h, pos.to(DEV), "k")
-        v = synth.key_values(spec, s, l, h, pos.to(DEV), "v")
-        kv.append(k)
-        vv.append(v)
-        rows_idx.append(np.full(count, r))
-        slots_all.append(slots)
-        pos_all.append(pos.numpy())
+        pos = torch.arange(n_total[s], n_total[s] + count, dtype=torch.int64, device=DEV)
+        kv[r] = synth.key_values(spec, s, l, h, pos, "k")
+        vv[r] = synth.key_values(spec, s, l, h, pos, "v")
         if r in states:
             st = states[r]
+            m = int(rl[r])
+            slots = np.arange(m, m + count)
             need = (m + count + P - 1) // P
             if st.kb.shape[0] < need:
                 extra = need - st.kb.shape[0]
                 st.kb = np.concatenate([st.kb, np.zeros((extra, P, D), dtype=st.kb.dtype)])
                 st.vb = np.concatenate([st.vb, np.zeros((extra, P, D), dtype=st.vb.dtype)])
-            st.kb.reshape(-1, D)[slots] = H._bits(k).cpu().numpy()
-            st.vb.reshape(-1, D)[slots] = H._bits(v).cpu().numpy()
-            st.sp[slots] = pos.numpy()
+            st.kb.reshape(-1, D)[slots] = H._bits(kv[r]).cpu().numpy()
+            st.vb.reshape(-1, D)[slots] = H._bits(vv[r]).cpu().numpy()
+            st.sp[slots] = pos.cpu().numpy()
             st.sl[slots] = synth.LABEL_REASON
             st.crf[slots] = 0.0
             st.n = m + count
-    ph = torch.from_numpy(np.concatenate(phys)).to(DEV)
-    c.k_pool.view(-1, D)[ph] = torch.cat(kv)
-    c.v_pool.view(-1, D)[ph] = torch.cat(vv)
-    ri = torch.from_numpy(np.concatenate(rows_idx)).to(DEV)
-    si = torch.from_numpy(np.concatenate(slots_all)).to(DEV)
-    c.slot_pos[ri, si] = torch.from_numpy(np.concatenate(pos_all).astype(np.int32)).to(DEV)
-    c.slot_label[ri, si] = synth.LABEL_REASON
-    rnd.crf[ri, si] = 0.0
-    c.block_table.copy_(torch.from_numpy(bt))
-    c.row_len.copy_(torch.from_numpy(rl + count))
+    ws = torch.zeros(kvc.kvc_append_workspace_bytes(spec.rows) // 8, dtype=torch.int64, device=DEV)
+    kvc.kvc_append_tokens(c, kv, vv, new_pos, synth.LABEL_REASON, rnd.crf, stack.pages, stack.depth, ws, rnd.status)
+    torch.cuda.synchronize()
+    assert rnd.device_status()[0] == 0, rnd.device_status()
+    assert np.array_equal(c.row_len.cpu().numpy(), rl + count)
     for s in range(spec.num_seqs):
         n_total[s] += count
 
@@ -254,7 +258,8 @@ def streaming_lockstep(spec, rounds, sample):
     computed by the library, the LRFU state carried across rounds, 64 decoded tokens appended after each
     compaction.  Every round compares the LSE, scores, kept set, CRF and the compacted row (pages bit for bit,
     positions, labels, freed pages); the oracle then carries on from the GPU's keep mask and, where a hit decision
-    sits in the gate-threshold band, from the GPU's CRF value, so that its state follows the GPU's."""
+    sits in the gate-threshold band, from the GPU's CRF value, so that its state follows the GPU's.  The decoded
+    tokens go in through the library's append (pages from a free stack fed by each compaction's freed list)."""
     w = H.build(spec)
     geo, P, G = w.geo, spec.page_size, spec.group
     rnd = EvictionRound(w.cache)
@@ -264,7 +269,7 @@ def streaming_lockstep(spec, rounds, sample):
               for r in sample}
     bt0 = w.cache.block_table.cpu().numpy()
     in_use = set(int(x) for x in bt0[bt0 >= 0])
-    free = [p for p in range(w.layout.num_pages) if p not in in_use]
+    stack = FreeStack([p for p in range(w.layout.num_pages) if p not in in_use], w.layout.num_pages)
     n_total = list(spec.ctx)
     band_total = 0
     for rd in range(rounds):
@@ -324,9 +329,9 @@ def streaming_lockstep(spec, rounds, sample):
             adopt = check_crf(gcrf, ocrf, osc, ohit, _orig_slots(src, dst, n), m, what)
             new.crf[:m][adopt] = gcrf[:m][adopt]
             st.kb, st.vb, st.sp, st.sl, st.crf, st.n = kb2[:kp], vb2[:kp], new.slot_pos, new.slot_label, new.crf, m
-        free.extend(int(x) for x in freed_dev)
+        stack.push(rnd.freed, nf)
         if rd + 1 < rounds:
-            append_tokens(w, rnd, n_total, free, states)
+            append_tokens(w, rnd, n_total, stack, states)
     return band_total
 
 
