@@ -162,9 +162,7 @@ kvc_status kvc_score_from_lse(const kvc_cache *cache, const kvc_queries *queries
     if (c.dtype == KVC_BF16 && !(flags & KVC_SCORE_SIMT)) {
         if (c.page_size != 16) return fail(KVC_ERR_UNSUPPORTED, "tensor-core scoring needs page_size 16");
         char err[256] = "";
-        cudaError_t e = kvc::score_pair_supported(c, q)
-                            ? kvc::launch_score_pair(c, q, scores, acc, d_status, st, err, sizeof(err))
-                            : kvc::launch_score_tc(c, q, scores, acc, d_status, st, err, sizeof(err));
+        cudaError_t e = kvc::launch_score_tc(c, q, scores, acc, d_status, st, err, sizeof(err));
         if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "score (tensor cores): %s %s", cudaGetErrorString(e), err);
         return KVC_OK;
     }

@@ -37,10 +37,6 @@ cudaError_t launch_score_simt(const CacheView &c, const QueryView &q, float *sco
 cudaError_t launch_lse_simt(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream);
 cudaError_t launch_score_tc(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
                             int32_t *status, cudaStream_t stream, char *err, size_t errlen);
-// Pair-of-SMs tensor-core scoring (bf16, head_dim 64 or 128, group size <= 128, query set within 256 blocks).
-bool score_pair_supported(const CacheView &c, const QueryView &q);
-cudaError_t launch_score_pair(const CacheView &c, const QueryView &q, float *scores, bool accumulate,
-                              int32_t *status, cudaStream_t stream, char *err, size_t errlen);
 // Tensor-core LSE pass (bf16, head_dim 64 or 128, group size <= 128).
 bool lse_tc_supported(const CacheView &c, const QueryView &q);
 cudaError_t launch_lse_tc(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream);

@@ -84,8 +84,8 @@ __device__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctrl &ctl, int32_t *sta
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = now_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 63) == 0) {
+        if (mbar_test_sleep(bar, parity, 20000u)) return true;
+        if ((it & 3) == 0) {
             if (*(volatile int32_t *)&ctl.abort) return false;
             if (now_ns() - t0 > kTimeoutNs) {
                 report(status, KVC_DEV_TIMEOUT, row);

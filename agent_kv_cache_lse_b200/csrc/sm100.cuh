@@ -1,7 +1,6 @@
-// Thin wrappers over the sm_100a instructions the tensor-core scoring kernel issues: mbarriers (local and
-// across the two CTAs of a cluster), tiled TMA loads, 5th-generation tensor-core MMAs with their
-// commit/fence operations, and TMEM loads.  Each wrapper is one instruction whose operand shapes the PTX ISA
-// fixes; none of them computes anything of the method.
+// Thin wrappers over the sm_100a instructions the tensor-core LSE pass issues: mbarriers, tiled TMA loads,
+// 5th-generation tensor-core MMAs with their commit/fence operations, and TMEM loads.  Each wrapper is one
+// instruction whose operand shapes the PTX ISA fixes; none of them computes anything of the method.
 #pragma once
 
 #include <cstdint>
@@ -18,23 +17,6 @@ __device__ __forceinline__ uint64_t now_ns() {
     return t;
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address of the same shared-memory location in the cluster CTA of rank `rank` (shared::cluster window).
-__device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -43,18 +25,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Arrive on a barrier given by its shared::cluster address (this CTA's or the peer's), release at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
-                 "r"(bytes)
-                 : "memory");
-}
-
-// Non-blocking test of a phase, with acquire at cluster scope (the arrivals may come from the peer CTA).
+// Non-blocking test of a phase (acquire: what the arrivals released is visible after it returns true).
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -67,24 +38,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Tiled TMA loads into this CTA's shared memory, completing bytes on a barrier given by its shared::cluster
-// address: with .cta_group::2 that barrier may be the peer CTA's (the pair's MMA waits on one barrier for the
-// operands of both CTAs).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+// As mbar_test, but a thread whose phase is not complete yet sleeps until it completes or about `hint_ns`
+// nanoseconds pass, instead of coming back at once (waiting warps then take no issue slots from working ones).
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
     asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z,
-                                                 int w) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-        "%5, %6}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
-        : "memory");
+    return ok != 0;
 }
 
 // Tiled TMA loads completing on a barrier of this CTA.
@@ -111,23 +76,12 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
 // fixed high word (stride byte offset, version, layout) and a low word holding the start address in 16-byte
 // units (14 bits) and the leading byte offset.
 constexpr uint32_t desc_hi(uint32_t sbo_bytes, uint32_t layout) { return (sbo_bytes >> 4) | (1u << 14) | (layout << 29); }
-constexpr uint32_t kLayoutSw128 = 2, kLayoutSw32 = 6;
+constexpr uint32_t kLayoutSw128 = 2;
 __device__ __forceinline__ uint32_t desc_lo(uint32_t addr) { return ((addr >> 4) & 0x3FFF) | (1u << 16); }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M x N.
 constexpr uint32_t idesc_bf16(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// One MMA of the CTA pair (issued by the even CTA): D[tmem] (+)= A * B^T, M = 256 rows split over the two CTAs'
-// shared memory (same address in both), B likewise split by columns.
-__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // One MMA of this CTA alone: D[tmem] (+)= A * B^T.
@@ -143,15 +97,6 @@ __device__ __forceinline__ void mma_cta(uint32_t d_tmem, uint64_t a_desc, uint64
 // Arrive once on this CTA's barrier when the MMAs this thread issued so far have completed.
 __device__ __forceinline__ void commit_cta(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// Arrive once on the barrier at this shared::cta offset in every CTA of `mask` when the pair's MMAs issued so far
-// have completed.
-__device__ __forceinline__ void commit_pair(uint64_t *bar, uint16_t mask) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-                     smem_u32(bar)),
-                 "h"(mask)
                  : "memory");
 }
 
@@ -180,53 +125,10 @@ __device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
-        "[%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-// Waits for this thread's TMEM loads; naming the registers of the load being waited for keeps the compiler from
-// reading them before the wait.
-__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
-                 :
-                 : "memory");
-}
-
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x on the FMA pipes for a pair of arguments: x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a degree-5
-// polynomial whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez exchange, derived by
-// exp2_poly.py beside this file: 2.4e-7 relative in fp32 Horner form, the accuracy class of the MUFU unit's
-// approximation, so that the two kinds of exponential are interchangeable under a 1e-4 ranking tolerance); 2^n
-// enters through the exponent bits.  x is clamped at -126 so the exponent arithmetic stays in range (the result is
-// then ~1e-38).  The floating-point steps run as packed f32x2 operations.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    constexpr float kC0 = 1.0000001192092896f, kC1 = 0.6931469440460205f, kC2 = 0.24022120237350464f,
-                    kC3 = 0.05550713092088699f, kC4 = 0.009675540961325169f, kC5 = 0.0013276472454890609f;
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
-    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-    const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-    float2 p = __ffma2_rn(make_float2(kC5, kC5), f, make_float2(kC4, kC4));
-    p = __ffma2_rn(p, f, make_float2(kC3, kC3));
-    p = __ffma2_rn(p, f, make_float2(kC2, kC2));
-    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace sm100
