@@ -229,6 +229,21 @@ kvc_status kvc_plan_slots(const kvc_cache *cache, const uint8_t *keep, const int
                        "kvc_plan_slots launch");
 }
 
+kvc_status kvc_select_plan(const kvc_cache *cache, const float *crf, const int32_t *budget,
+                           uint32_t protect_label_mask, uint8_t *keep, int32_t *kept, int32_t *move_src,
+                           int32_t *move_dst, int32_t *num_moves, int32_t *d_status, kvc_stream_t stream) {
+    g_err[0] = 0;
+    kvc::CacheView c;
+    kvc_status s = view_cache(cache, c, false);
+    if (s != KVC_OK) return s;
+    if (!crf || !budget || !keep || !kept) return fail(KVC_ERR_INVALID_ARGUMENT, "crf, budget, keep and kept are required");
+    if (!move_src || !move_dst || !num_moves)
+        return fail(KVC_ERR_INVALID_ARGUMENT, "move_src, move_dst and num_moves are required");
+    return cuda_status(kvc::launch_select_plan(c, crf, budget, protect_label_mask, keep, kept, move_src, move_dst,
+                                               num_moves, d_status, (cudaStream_t)stream),
+                       "kvc_select_plan launch");
+}
+
 size_t kvc_compact_workspace_bytes(int32_t rows) {
     return rows < 0 ? 0 : ((size_t)rows + 1) * sizeof(int64_t);
 }

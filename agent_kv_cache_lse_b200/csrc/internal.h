@@ -49,6 +49,9 @@ cudaError_t launch_lrfu_select(const CacheView &c, const float *scores, float *c
                                int32_t *status, cudaStream_t stream);
 cudaError_t launch_plan(const CacheView &c, const uint8_t *keep, const int32_t *kept, int32_t *move_src,
                         int32_t *move_dst, int32_t *num_moves, int32_t *status, cudaStream_t stream);
+cudaError_t launch_select_plan(const CacheView &c, const float *crf, const int32_t *budget, uint32_t protect,
+                               uint8_t *keep, int32_t *kept, int32_t *move_src, int32_t *move_dst,
+                               int32_t *num_moves, int32_t *status, cudaStream_t stream);
 cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const int32_t *move_dst,
                            const int32_t *num_moves, const int32_t *new_len, float *crf, int32_t *freed,
                            int64_t freed_capacity, int64_t *num_freed, int64_t *row_offsets,

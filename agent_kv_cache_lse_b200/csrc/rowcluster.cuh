@@ -20,6 +20,7 @@ namespace kvc {
 namespace cg = cooperative_groups;
 
 constexpr int kRowBins = 256;  // 8-bit digits, 4 passes over 32-bit keys
+constexpr int kRowCand = 256;  // a search whose current bin holds at most this many entries finishes on them
 
 // Per-CTA histogram of one digit.  A mass is a fixed-point integer below 2^48, kept as three 16-bit
 // chunks summed in 32-bit counters (a CTA's slice holds at most 65,536 entries, so no chunk sum can
@@ -45,6 +46,16 @@ struct RowShared {
     int red_i[32];
     unsigned long long red_u[32];
     float red_f[32];
+    // candidate finish: this CTA's entries of the search's current bin (published to the cluster), and every
+    // CTA's gathered copy of all of them
+    unsigned int ncand;
+    unsigned int cn[8], cb[9];          // every rank's count, gathered, and their prefix sums
+    uint32_t ck[kRowCand];
+    unsigned long long cw[kRowCand];
+    uint32_t gk[kRowCand];
+    unsigned long long gw[kRowCand];
+    uint32_t fin_key, fin_eq;
+    unsigned long long fin_above;
 };
 
 struct RowCtx {
@@ -133,6 +144,82 @@ __device__ inline unsigned long long row_sum_u64(RowCtx &rc, RowShared &sh, unsi
     for (int r = 0; r < rc.nranks; ++r) tot += rc.cl.map_shared_rank(&sh, r)->xu[b];
     rc.par++;
     return tot;
+}
+
+// End of a mass-weighted radix search once the current bin (keys matching sh.prefix under sh.pmask) holds at
+// most kRowCand valid entries cluster-wide: every CTA lists its entries of the bin, the cluster barrier publishes the lists,
+// and every CTA gathers all of them (rank order) and finds the threshold itself: the key T whose weight
+// interval (above(T), above(T) + weight(== T)] in descending key order holds the remaining target.  Each
+// entry's interval is found by one pass over the gathered list (at most kRowCand x kRowCand steps), so the
+// result is exact and the same in every CTA.  Saves the remaining radix passes (each a sweep, a barrier and
+// a gather of four histograms).
+template <bool kMass, typename KeyFn, typename WeightFn, typename ValidFn>
+__device__ void row_finish_candidates(RowCtx &rc, RowShared &sh, int lo, int hi, KeyFn key, WeightFn weight,
+                                      ValidFn valid) {
+    const int tid = threadIdx.x;
+    const uint32_t prefix = sh.prefix, pmask = sh.pmask;
+    if (tid == 0) sh.ncand = 0;
+    __syncthreads();
+    for (int i = lo + tid; i < hi; i += blockDim.x) {
+        if (!valid(i)) continue;
+        const uint32_t k = key(i);
+        if ((k & pmask) != prefix) continue;
+        const unsigned at = atomicAdd(&sh.ncand, 1u);   // below kRowCand: the bin's count bounds it
+        sh.ck[at] = k;
+        sh.cw[at] = kMass ? (unsigned long long)weight(i) : 1ull;
+    }
+    rc.cl.sync();
+    // the ranks' counts first (one remote load each, side by side), then every entry of every rank, each thread
+    // loading its share with all its loads in flight
+    if (tid < rc.nranks) sh.cn[tid] = rc.cl.map_shared_rank(&sh, tid)->ncand;
+    __syncthreads();
+    if (tid == 0) {
+        unsigned int b = 0;
+        for (int r = 0; r < rc.nranks; ++r) {
+            sh.cb[r] = b;
+            b += sh.cn[r];
+        }
+        sh.cb[rc.nranks] = b;
+    }
+    __syncthreads();
+    const int nc = (int)sh.cb[rc.nranks];
+    for (int e = tid; e < rc.nranks * kRowCand; e += blockDim.x) {
+        const int r = e / kRowCand, j = e % kRowCand;
+        if (j < (int)sh.cn[r]) {
+            const RowShared *p = rc.cl.map_shared_rank(&sh, r);
+            sh.gk[sh.cb[r] + j] = p->ck[j];
+            sh.gw[sh.cb[r] + j] = p->cw[j];
+        }
+    }
+    __syncthreads();
+    const unsigned long long rem = sh.remaining;
+    for (int i = tid; i < nc; i += blockDim.x) {
+        const uint32_t ki = sh.gk[i];
+        unsigned long long above = 0, eqw = 0;
+        uint32_t eqc = 0;
+        for (int j = 0; j < nc; ++j) {
+            const uint32_t kj = sh.gk[j];
+            const unsigned long long w = sh.gw[j];
+            if (kj > ki) {
+                above += w;
+            } else if (kj == ki) {
+                eqw += w;
+                ++eqc;
+            }
+        }
+        if (above < rem && rem <= above + eqw) {   // one key qualifies; its copies write the same values
+            sh.fin_key = ki;
+            sh.fin_above = above;
+            sh.fin_eq = eqc;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        sh.prefix = sh.fin_key;
+        sh.above += sh.fin_above;
+        sh.eq_count = sh.fin_eq;
+    }
+    __syncthreads();
 }
 
 // Radix search over the cluster's row, from the most significant 8-bit digit down.  Finds the key T
@@ -265,6 +352,10 @@ __device__ RadixResult row_radix_desc(RowCtx &rc, RowShared &sh, int lo, int hi,
             }
         }
         __syncthreads();
+        if (kMass && pass < 3 && sh.eq_count <= (uint32_t)kRowCand) {   // (count passes are cheaper than the finish)
+            row_finish_candidates<kMass>(rc, sh, lo, hi, key, weight, valid);
+            break;
+        }
     }
     RadixResult r;
     r.key = sh.prefix;

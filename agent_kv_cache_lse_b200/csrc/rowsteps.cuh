@@ -1,6 +1,6 @@
-// Per-row bodies of the LRFU update and the top-budget selection, shared by their own kernels and by the
-// fused kernel that runs both in one launch.  Each body is one CTA's part of a cluster that shares a row
-// (rowcluster.cuh); the fused kernel calls them back to back with the same cluster context.
+// Per-row bodies of the LRFU update, the top-budget selection and the slot plan, shared by their own kernels
+// and by the fused kernels that run two of them in one launch.  Each body is one CTA's part of a cluster that
+// shares a row (rowcluster.cuh); a fused kernel calls them back to back with the same cluster context.
 #pragma once
 
 #include "internal.h"
@@ -20,6 +20,16 @@ struct LrfuArgs {
     int32_t *status;
     int slice_cap;    // scores cached in shared memory when a CTA's slice fits
     int weight_cap;   // fixed-point masses cached too when the slice fits this
+};
+
+struct PlanArgs {
+    CacheView c;
+    const uint8_t *keep;
+    const int32_t *kept;
+    int32_t *move_src;
+    int32_t *move_dst;
+    int32_t *num_moves;
+    int32_t *status;
 };
 
 struct SelectArgs {
@@ -273,5 +283,64 @@ __device__ inline void select_row(const SelectArgs &a, RowCtx &rc, unsigned char
     rc.cl.sync();
 }
 
+
+
+// Conflict-free slot plan of this CTA's slice of its row ("ActKV Dissected", Component 3): survivor j at or
+// after m = kept (ascending) fills hole j before m (ascending).  Every thread owns a contiguous run of slots; a
+// CTA scan plus the cluster-wide sums of the lower slices give every hole and survivor its rank, its index in
+// the move list.  A rejected row gets num_moves = -1, which the compaction reads as "leave this row as it is".
+__device__ inline void plan_row(const PlanArgs &a, RowCtx &rc, RowShared &sh) {
+    const int row = blockIdx.x / rc.nranks;
+    const CacheView &c = a.c;
+    const int n = c.row_len[row];
+    const int m = a.kept[row];
+    if (n < 0 || n > c.max_slots || m < 0 || m > n) {
+        if (rc.rank == 0 && threadIdx.x == 0) {
+            a.num_moves[row] = -1;
+            report(a.status, (n < 0 || n > c.max_slots) ? KVC_DEV_BAD_LENGTH : KVC_DEV_KEPT_MISMATCH, row);
+        }
+        return;  // uniform across the cluster: no collective has started
+    }
+    const int per = (n + rc.nranks - 1) / rc.nranks;
+    const int lo = min(n, rc.rank * per), hi = min(n, lo + per);
+    const uint8_t *keep = a.keep + (int64_t)row * c.max_slots;
+    const int span = hi - lo;
+    const int chunk = (span + blockDim.x - 1) / blockDim.x;
+    const int b0 = lo + min(span, (int)threadIdx.x * chunk), b1 = lo + min(span, ((int)threadIdx.x + 1) * chunk);
+    int holes = 0, movers = 0;
+    for (int i = b0; i < b1; ++i) {
+        const int k = keep[i] != 0;
+        if (i < m) holes += !k;
+        else movers += k;
+    }
+    int th, tm;
+    int hr = block_exclusive_scan(holes, sh.red_i, &th);
+    int mr = block_exclusive_scan(movers, sh.red_i, &tm);
+    int tot[2], below[2];
+    row_sum_int2(rc, sh, holes, movers, tot, below);
+    // kept count consistent with the mask  <=>  as many holes before m as survivors after it
+    if (tot[0] != tot[1]) {
+        if (rc.rank == 0 && threadIdx.x == 0) {
+            a.num_moves[row] = -1;
+            report(a.status, KVC_DEV_KEPT_MISMATCH, row);
+        }
+        rc.cl.sync();
+        return;
+    }
+    hr += below[0];
+    mr += below[1];
+    int32_t *src = a.move_src + (int64_t)row * c.max_slots;
+    int32_t *dst = a.move_dst + (int64_t)row * c.max_slots;
+    for (int i = b0; i < b1; ++i) {
+        const int k = keep[i] != 0;
+        if (i < m) {
+            if (!k) dst[hr++] = i;
+        } else if (k) {
+            src[mr++] = i;
+        }
+    }
+    if (rc.rank == 0 && threadIdx.x == 0) a.num_moves[row] = tot[0];
+    rc.cl.sync();
+}
 
 }  // namespace kvc

@@ -29,7 +29,7 @@ EXPORTS = ["kvc_status_string", "kvc_last_error", "kvc_version", "kvc_query_lse"
            "kvc_lrfu_update", "kvc_select_budget", "kvc_plan_slots", "kvc_compact_workspace_bytes",
            "kvc_compact_pages", "kvc_compact_pages_noalloc", "kvc_ratchet_state_bytes", "kvc_ratchet_init",
            "kvc_confidence_ratchet", "kvc_beacon_update", "kvc_lrfu_select", "kvc_decode_attention",
-           "kvc_step_scores", "kvc_append_workspace_bytes", "kvc_append_tokens"]
+           "kvc_step_scores", "kvc_append_workspace_bytes", "kvc_append_tokens", "kvc_select_plan"]
 
 
 class KvcCache(ctypes.Structure):
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
             "kvc_select_budget": (ctypes.c_int, [pc, vp, vp, u32, vp, vp, vp, vp]),
             "kvc_lrfu_select": (ctypes.c_int, [pc, vp, vp, f32, f32, i32, u32, vp, u32, vp, vp, vp, vp]),
             "kvc_plan_slots": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, vp]),
+            "kvc_select_plan": (ctypes.c_int, [pc, vp, vp, u32, vp, vp, vp, vp, vp, vp, vp]),
             "kvc_compact_workspace_bytes": (ctypes.c_size_t, [i32]),
             "kvc_compact_pages": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, i64, vp, vp, ctypes.c_size_t, vp, vp]),
             "kvc_compact_pages_noalloc": (ctypes.c_int, [pc, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp]),
@@ -229,6 +230,16 @@ def kvc_plan_slots(cache: Cache, keep: torch.Tensor, kept: torch.Tensor, move_sr
     cs = cache.struct()
     _check(lib().kvc_plan_slots(ctypes.byref(cs), _ptr(keep), _ptr(kept), _ptr(move_src), _ptr(move_dst),
                                 _ptr(num_moves), _ptr(d_status), _stream(stream)), "kvc_plan_slots")
+
+
+def kvc_select_plan(cache: Cache, crf: torch.Tensor, budget: torch.Tensor, keep: torch.Tensor, kept: torch.Tensor,
+                    move_src: torch.Tensor, move_dst: torch.Tensor, num_moves: torch.Tensor,
+                    protect_label_mask: int = 0, d_status=None, stream=None):
+    """kvc_select_budget followed by kvc_plan_slots, in one launch."""
+    cs = cache.struct()
+    _check(lib().kvc_select_plan(ctypes.byref(cs), _ptr(crf), _ptr(budget), protect_label_mask, _ptr(keep), _ptr(kept),
+                                 _ptr(move_src), _ptr(move_dst), _ptr(num_moves), _ptr(d_status), _stream(stream)),
+           "kvc_select_plan")
 
 
 def kvc_compact_workspace_bytes(rows: int) -> int:

@@ -69,8 +69,8 @@ class EvictionRound:
 
     def run_after_scores(self, logits: Optional[torch.Tensor], lam: float = 0.5, hit_mass: float = 0.9, stream=None,
                          protect_label_mask: int = 0, confidence_out: Optional[torch.Tensor] = None):
-        """Enqueue the rest of a round on scores already in self.scores: (ratchet | LRFU) -> select -> plan ->
-        compact, or LRFU + select in one launch when there are no logits."""
+        """Enqueue the rest of a round on scores already in self.scores: (ratchet | LRFU) -> select + plan (one
+        launch) -> compact, or LRFU + select (one launch) -> plan -> compact when there are no logits."""
         c = self.cache
         main = stream if stream is not None else torch.cuda.current_stream()
         if logits is not None:
@@ -82,11 +82,13 @@ class EvictionRound:
                                        self._side)
             self._join.record(self._side)
             main.wait_event(self._join)
-            kvc.kvc_select_budget(c, self.crf, self.budget, self.keep, self.kept, protect_label_mask, self.status, main)
+            kvc.kvc_select_plan(c, self.crf, self.budget, self.keep, self.kept, self.move_src, self.move_dst,
+                                self.num_moves, protect_label_mask, self.status, main)
         else:
             kvc.kvc_lrfu_select(c, self.scores, self.crf, self.budget, self.keep, self.kept, lam, hit_mass, 1, 0,
                                 protect_label_mask, self.status, main)
-        kvc.kvc_plan_slots(c, self.keep, self.kept, self.move_src, self.move_dst, self.num_moves, self.status, main)
+            kvc.kvc_plan_slots(c, self.keep, self.kept, self.move_src, self.move_dst, self.num_moves, self.status,
+                               main)
         kvc.kvc_compact_pages(c, self.move_src, self.move_dst, self.num_moves, self.kept, self.crf, self.freed,
                               self.num_freed, self.workspace, self.status, main)
 

@@ -211,7 +211,7 @@ def run_ours(args, rank, world, device):
     fork, join = torch.cuda.Event(), torch.cuda.Event()
 
     def step(e=None):
-        # score, then the ratchet (side stream) beside the LRFU update, then select, plan, compact
+        # score, then the ratchet (side stream) beside the LRFU update, then select + plan (one launch), compact
         main = torch.cuda.current_stream()
         if e is not None:
             e[0].record(main)
@@ -227,8 +227,8 @@ def run_ours(args, rank, world, device):
             e[2].record(side)
         join.record(side)
         main.wait_event(join)
-        kvc.kvc_select_budget(cache, rnd.crf, rnd.budget, rnd.keep, rnd.kept, 0, rnd.status, main)
-        kvc.kvc_plan_slots(cache, rnd.keep, rnd.kept, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.status, main)
+        kvc.kvc_select_plan(cache, rnd.crf, rnd.budget, rnd.keep, rnd.kept, rnd.move_src, rnd.move_dst,
+                            rnd.num_moves, 0, rnd.status, main)
         kvc.kvc_compact_pages(cache, rnd.move_src, rnd.move_dst, rnd.num_moves, rnd.kept, rnd.crf, rnd.freed,
                               rnd.num_freed, rnd.workspace, rnd.status, main)
         if e is not None:
@@ -334,7 +334,7 @@ def run_ours(args, rank, world, device):
     return line
 
 
-EvictionRound_KERNELS = 8
+EvictionRound_KERNELS = 7   # score, LRFU, confidence, ratchet update, select + plan, compaction moves, freed pages
 
 SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_batch16_layer.md")

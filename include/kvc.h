@@ -246,6 +246,18 @@ kvc_status kvc_plan_slots(const kvc_cache *cache, const uint8_t *keep, const int
                           int32_t *move_src, int32_t *move_dst, int32_t *num_moves,
                           int32_t *d_status, kvc_stream_t stream);
 
+/*
+ * kvc_select_budget followed by kvc_plan_slots, in one launch: the same arguments, checks,
+ * device errors and results (keep, kept, move_src, move_dst, num_moves) as the two calls in
+ * sequence, with the plan reading the keep mask and kept counts this launch has just written.
+ * (A system-level fusion of two steps of "ActKV Dissected", Summary and Component 3; the pages
+ * have no counterpart of the entry point itself.)
+ */
+kvc_status kvc_select_plan(const kvc_cache *cache, const float *crf, const int32_t *budget,
+                           uint32_t protect_label_mask, uint8_t *keep, int32_t *kept,
+                           int32_t *move_src, int32_t *move_dst, int32_t *num_moves,
+                           int32_t *d_status, kvc_stream_t stream);
+
 /* bytes of device workspace kvc_compact_pages needs for `rows` rows */
 size_t kvc_compact_workspace_bytes(int32_t rows);
 

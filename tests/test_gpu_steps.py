@@ -256,6 +256,44 @@ def test_lrfu_select_fused_matches_separate(mode):
         assert np.array_equal(k1[r, :n].astype(bool), ok), f"row {r}"
 
 
+@pytest.mark.parametrize("mode", ["lognormal", "ties", "equal"])
+def test_select_plan_fused_matches_separate(mode):
+    """kvc_select_plan equals kvc_select_budget then kvc_plan_slots: the same keep mask, counts, move lists and
+    move counts, with protected labels; and the plan it makes equals the oracle's on that mask."""
+    rng = np.random.default_rng(43)
+    lengths = [0, 1, 16, 257, 5000, 33000]
+    ms = 33008
+    c = bare_cache(lengths, ms, S=len(lengths))
+    crf0 = np.zeros((len(lengths), ms), dtype=np.float32)
+    for r, n in enumerate(lengths):
+        crf0[r, :n] = _row_values(rng, n, mode)
+    budgets = torch.tensor([3, 0, 5, 100, 512, 2048], dtype=torch.int32, device=DEV)
+    crf = torch.from_numpy(crf0).to(DEV)
+    outs = []
+    for fused in (False, True):
+        keep = torch.full((len(lengths), ms), 9, dtype=torch.uint8, device=DEV)
+        kept = torch.zeros(len(lengths), dtype=torch.int32, device=DEV)
+        src = torch.full((len(lengths), ms), -7, dtype=torch.int32, device=DEV)
+        dst = torch.full((len(lengths), ms), -7, dtype=torch.int32, device=DEV)
+        nm = torch.full((len(lengths),), -7, dtype=torch.int32, device=DEV)
+        st = torch.zeros(2, dtype=torch.int32, device=DEV)
+        if fused:
+            kvc.kvc_select_plan(c, crf, budgets, keep, kept, src, dst, nm, 1 << 2, st)
+        else:
+            kvc.kvc_select_budget(c, crf, budgets, keep, kept, 1 << 2, st)
+            kvc.kvc_plan_slots(c, keep, kept, src, dst, nm, st)
+        torch.cuda.synchronize()
+        outs.append([t.cpu().numpy() for t in (keep, kept, src, dst, nm)] + [st.cpu().tolist()])
+    for a, b in zip(outs[0][:5], outs[1][:5]):
+        assert np.array_equal(a, b)
+    assert outs[0][5] == outs[1][5] == [0, 0]
+    keep, kept, src, dst, nm = outs[1][:5]
+    for r, n in enumerate(lengths):
+        want_src, want_dst, m = opath.plan_slots(keep[r, :n].astype(bool), n)
+        assert int(nm[r]) == len(want_src) and int(kept[r]) == m
+        assert np.array_equal(src[r, :len(want_src)], want_src) and np.array_equal(dst[r, :len(want_dst)], want_dst)
+
+
 def _masks(rng, lengths, mode):
     keeps = []
     for n in lengths:
