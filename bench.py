@@ -242,7 +242,7 @@ def run_ours(args, rank, world, device):
     if code != 0:
         raise RuntimeError(f"device status {rnd.device_status()} during warm-up")
 
-    # the round as one CUDA graph (six calls, eight kernels, the ratchet on a parallel branch), with timing
+    # the round as one CUDA graph (five calls, seven kernels, the ratchet on a parallel branch), with timing
     # events captured as nodes
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     graph = None
@@ -334,7 +334,7 @@ def run_ours(args, rank, world, device):
     return line
 
 
-EvictionRound_KERNELS = 7   # score, LRFU, confidence, ratchet update, select + plan, compaction moves, freed pages
+EvictionRound_KERNELS = 7   # score, LRFU, confidence, budget update, select + plan, compaction moves, freed pages
 
 SCORE_PROFILE = os.path.join(ROOT, "profiles", "score_tc_llama8b_32k.md")
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_batch16_layer.md")
@@ -1145,7 +1145,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
-    ap.add_argument("--no-graph", action="store_true", help="launch the six calls directly instead of a CUDA graph")
+    ap.add_argument("--no-graph", action="store_true", help="launch the round's five calls directly instead of a CUDA graph")
     ap.add_argument("--beacon", action="store_true", help="time beacon-query maintenance instead of the round")
     ap.add_argument("--decode", action="store_true", help="time the fused decode step instead of the round")
     ap.add_argument("--stepkv", action="store_true", help="time the step-aware ranking scores instead of the round")
