@@ -136,8 +136,7 @@ cudaError_t launch_append(const CacheView &c, const void *k_new, const void *v_n
     append_plan_kernel<<<1, kThreads, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms();
     const int per_row_warps = (count + 7) / 8;
     const int xb = std::max(1, std::min(std::max(1, (4 * sms + c.rows - 1) / c.rows), per_row_warps));
     append_write_kernel<<<dim3(xb, c.rows), kThreads, 0, stream>>>(a);

@@ -223,7 +223,8 @@ cudaError_t launch_beacon(const void *q, const int32_t *num_q, int32_t num_seqs,
     rows = std::max(rows, round_rows);
     const size_t smem = fixed + (size_t)rows * (head_dim + 1) * 4;
     if (smem > kSmemCap - 2048) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(beacon_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)beacon_kernel, smem, smem_set);
     if (e != cudaSuccess) return e;
     BeaconArgs a{q, num_q, num_layers, num_q_heads, head_dim, max_q, bf16 ? 1 : 0, beacons, counts, num_beacons,
                  beacon_q, out_max_q, rows, status};

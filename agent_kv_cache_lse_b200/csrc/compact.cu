@@ -151,9 +151,7 @@ cudaError_t launch_compact(const CacheView &c, const int32_t *move_src, const in
     const int esize = c.dtype == KVC_BF16 ? 2 : 4;
     CompactArgs a{c, move_src, move_dst, num_moves, new_len, crf, freed, freed_capacity, num_freed,
                   row_offsets, status, c.head_dim * esize / 16};
-    int sms = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms();
     const int xa = std::max(1, std::min(64, (4 * sms + c.rows - 1) / c.rows));
     compact_moves_kernel<<<dim3(xa, c.rows + 1), kThreads, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();

@@ -548,19 +548,14 @@ Plan plan_for(const CacheView &c, int G, int sms) {
     return Plan{};
 }
 
-int sm_count() {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return sms;
-}
+int sm_count() { return device_sms(); }
 
 template <typename T, int D, int GM, int RW>
 cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                      float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, const Plan &p) {
     const int G = num_q_heads / c.num_kv_heads;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D, GM, RW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)p.smem);
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)decode_kernel<T, D, GM, RW>, p.smem, smem_set);
     if (e != cudaSuccess) return e;
     DecodeArgs a{c, q, q_pos, num_q_heads, G, out, lse, scores, accumulate ? 1 : 0, p.CH, p.RW, p.cap,
                  (float)(1.4426950408889634 / std::sqrt((double)D)), status};

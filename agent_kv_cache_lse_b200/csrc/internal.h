@@ -8,6 +8,37 @@
 
 namespace kvc {
 
+// Host-side lookups done once per device instead of on every call.
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device.
+inline int device_sms() {
+    static int cache[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    int &v = cache[dev & (kMaxDevices - 1)];
+    if (v == 0) {
+        int sms = 148;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) v = sms;
+        else return sms;
+    }
+    return v;
+}
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device; `done` (one array per
+// kernel, kMaxDevices entries, zero-initialised) remembers what each device was given, so the attribute is set
+// only when a call needs more than before.
+inline cudaError_t dyn_smem_at_least(const void *kernel, size_t bytes, int *done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int &have = done[dev & (kMaxDevices - 1)];
+    if ((size_t)have >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) have = (int)bytes;
+    return e;
+}
+
 // Geometry and pointers resolved once on the host for a call.
 struct CacheView {
     const void *k_pool;

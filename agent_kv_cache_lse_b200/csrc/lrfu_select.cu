@@ -21,9 +21,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) lrfu_select_kernel(LrfuArgs la
 cudaError_t launch_lrfu_select(const CacheView &c, const float *scores, float *crf, float decay, float hit_mass,
                                bool binary, const int32_t *budget, uint32_t protect, uint8_t *keep, int32_t *kept,
                                int32_t *status, cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms();
     int C = row_cluster_size(c.rows, sms);
     while (C < 8 && (c.max_slots + C - 1) / C > 65536) C <<= 1;  // the mass chunks need slices of at most 2^16
     if ((c.max_slots + C - 1) / C > 65536) return cudaErrorInvalidValue;
@@ -31,7 +29,8 @@ cudaError_t launch_lrfu_select(const CacheView &c, const float *scores, float *c
     const int cap = per < 40960 ? per : 0;
     const int wcap = cap > 0 && per <= 12288 ? per : 0;
     const size_t smem = sizeof(RowShared) + (((size_t)cap * 4 + 15) & ~(size_t)15) + (size_t)wcap * 8;
-    cudaError_t e = cudaFuncSetAttribute(lrfu_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)lrfu_select_kernel, smem, smem_set);
     if (e != cudaSuccess) return e;
     LrfuArgs la{c, scores, crf, decay, hit_mass, binary ? 1 : 0, status, cap, wcap};
     SelectArgs sa{c, crf, budget, protect, keep, kept, status, cap};

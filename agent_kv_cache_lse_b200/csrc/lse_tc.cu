@@ -393,8 +393,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_lse() {
     return fn;
 }
 
-bool g_lse_attr[64][2];
-
 template <int D>
 cudaError_t launch_lse_tc_t(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream) {
     using PL = LPlan<D>;
@@ -431,14 +429,9 @@ cudaError_t launch_lse_tc_t(const CacheView &c, const QueryView &q, int32_t *sta
     args.nqt = nqt;
     args.tiles_q = (q.max_q + nqt - 1) / nqt;
     args.scale_log2e = (float)(1.4426950408889634 / std::sqrt((double)D));
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)lse_tc_kernel<D>, PL::kBytes, smem_set);
     if (e != cudaSuccess) return e;
-    if (!g_lse_attr[dev & 63][D == 128]) {
-        e = cudaFuncSetAttribute(lse_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
-        if (e != cudaSuccess) return e;
-        g_lse_attr[dev & 63][D == 128] = true;
-    }
     const int64_t grid = (int64_t)c.rows * args.tiles_q;
     if (grid <= 0) return cudaSuccess;
     lse_tc_kernel<D><<<(unsigned)grid, kThreads, PL::kBytes, stream>>>(tk, tq, args);

@@ -27,9 +27,7 @@ __global__ void __launch_bounds__(kThreads) plan_kernel(PlanArgs a) {
 
 cudaError_t launch_plan(const CacheView &c, const uint8_t *keep, const int32_t *kept, int32_t *move_src,
                         int32_t *move_dst, int32_t *num_moves, int32_t *status, cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms();
     const int C = row_cluster_size(c.rows, sms);
     PlanArgs a{c, keep, kept, move_src, move_dst, num_moves, status};
     cudaLaunchConfig_t cfg = {};

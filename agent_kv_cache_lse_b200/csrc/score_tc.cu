@@ -1093,10 +1093,9 @@ cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool
     args.tiles_per_row = (int)((c.max_slots + kTileKeys - 1) / kTileKeys);
     args.total_tiles = (int64_t)c.rows * args.tiles_per_row;
     args.scale_log2e = (float)(1.4426950408889634 / std::sqrt((double)D));
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
+    const int sms = device_sms();
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)score_tc_kernel<D>, PL::kBytes, smem_set);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<int64_t>(sms, args.total_tiles);
     score_tc_kernel<D><<<grid, kThreads, PL::kBytes, stream>>>(tk, tq, args);

@@ -24,14 +24,13 @@ __global__ void __launch_bounds__(kRowThreads, 1) select_kernel(SelectArgs a) {
 
 cudaError_t launch_select(const CacheView &c, const float *crf, const int32_t *budget, uint32_t protect,
                           uint8_t *keep, int32_t *kept, int32_t *status, cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sms();
     const int C = row_cluster_size(c.rows, sms);
     const int per = (int)((c.max_slots + C - 1) / C);
     const int cap = per < 40960 ? per : 0;
     const size_t smem = sizeof(RowShared) + (size_t)cap * 4;
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_set[kMaxDevices];
+    cudaError_t e = dyn_smem_at_least((const void *)select_kernel, smem, smem_set);
     if (e != cudaSuccess) return e;
     SelectArgs a{c, crf, budget, protect, keep, kept, status, cap};
     cudaLaunchConfig_t cfg = {};

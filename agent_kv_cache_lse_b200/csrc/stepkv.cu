@@ -265,8 +265,8 @@ cudaError_t launch_step_scores(const CacheView &c, const float *scores, const in
                                cudaStream_t stream) {
     if (c.max_slots <= (int64_t)kRegThreads * kRegSlots && max_steps <= 65536) {
         const size_t smem = (size_t)max_steps * (8 + 4 + 4) + (size_t)kRegThreads * kRegSlots * 2;
-        cudaError_t e = cudaFuncSetAttribute(step_scores_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        static int smem_set[kMaxDevices];
+        cudaError_t e = dyn_smem_at_least((const void *)step_scores_reg_kernel, smem, smem_set);
         if (e != cudaSuccess) return e;
         step_scores_reg_kernel<<<c.rows, kRegThreads, smem, stream>>>(
             StepArgs{c, scores, step_start, num_steps, max_steps, beta, out, status});
@@ -274,7 +274,8 @@ cudaError_t launch_step_scores(const CacheView &c, const float *scores, const in
     }
     const size_t smem = (size_t)max_steps * (8 + 4 + 4);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(step_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static int smem_set[kMaxDevices];
+        cudaError_t e = dyn_smem_at_least((const void *)step_scores_kernel, smem, smem_set);
         if (e != cudaSuccess) return e;
     }
     step_scores_kernel<<<c.rows, kThreads, smem, stream>>>(
