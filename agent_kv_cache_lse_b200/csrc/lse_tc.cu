@@ -6,11 +6,13 @@
 //
 //   lse[seq][layer][h][j] = ln sum_{i : slot_pos_i <= q_pos_j} exp(q_{j,h} . k_i / sqrt(D))      (-inf: no key)
 //
-// CTA per (row, tile of 128 query columns: floor(128 / G) queries x G heads, query-major); the CTA's columns
-// stay in shared memory (the A operand) while the row's keys stream through in tiles of 128 (the B operand,
-// gathered page by page with TMA).  One M128 x N128 x K=D tcgen05.mma per key tile into one of four TMEM
+// A cluster of S CTAs per (row, tile of 128 query columns: floor(128 / G) queries x G heads, query-major), each
+// CTA a contiguous share of the row's key tiles (S is chosen on the host so the CTAs fill whole waves of SMs);
+// the CTA's columns stay in shared memory (the A operand) while its keys stream through in tiles of 128 (the B
+// operand, gathered page by page with TMA).  One M128 x N128 x K=D tcgen05.mma per key tile into one of four TMEM
 // accumulators; 16 epilogue warps (TMEM lane quadrant = 32 columns, key quarter = 32 keys of the tile) keep a
-// running (max, sum) per column in the log2 domain, merged over the quarters at the end.
+// running (max, sum) per column in the log2 domain, merged over the quarters at the end, then over the
+// cluster's CTAs through distributed shared memory.
 //   warp 0  TMA: the query tile once, then per key tile its 8 pages (16 x 64 bf16 boxes, 128B swizzle).
 //   warp 1  TMEM owner and MMA issuer.
 //   warp 2  key decoder: per key tile the pages and the slot positions (readable keys only).
@@ -24,9 +26,13 @@
 #include <cmath>
 #include <cstdio>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace kvc {
 namespace {
@@ -56,6 +62,7 @@ struct Ctrl {
     uint32_t tmem_base;
     int32_t abort;
     float part_m[3][kCols], part_s[3][kCols];
+    float fin_m[kCols], fin_s[kCols];     // this CTA's (max, sum) per column when a row's keys are split
 };
 
 struct LseTcArgs {
@@ -64,6 +71,7 @@ struct LseTcArgs {
     int32_t *status;
     int nqt;           // queries per CTA tile: floor(128 / G)
     int tiles_q;       // column tiles per row
+    int splits;        // CTAs (one cluster) sharing a column tile, each a contiguous run of the row's key tiles
     float scale_log2e; // log2(e) / sqrt(D)
 };
 
@@ -109,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const CacheView &c = a.c;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x / a.tiles_q, qt = blockIdx.x % a.tiles_q;
+    const int split = blockIdx.x % a.splits, unit = blockIdx.x / a.splits;
+    const int row = unit / a.tiles_q, qt = unit % a.tiles_q;
     const int RPS = c.num_layers * c.num_kv_heads;
     const int seq = row / RPS, layer = (row / c.num_kv_heads) % c.num_layers, kvh = row % c.num_kv_heads;
     const int G = a.q.group, nqt = a.nqt;
@@ -123,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (n == 0) {
         // no keys: every column of the tile sees nothing
-        for (int col = threadIdx.x; col < nqt * G; col += kThreads) {
+        for (int col = threadIdx.x; split == 0 && col < nqt * G; col += kThreads) {
             const int j = j0 + col / G;
             if (j < nq)
                 a.q.lse[((int64_t)(seq * c.num_layers + layer) * a.q.num_q_heads + kvh * G + col % G) * a.q.max_q + j] =
@@ -167,17 +176,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
     const int ntiles = (n + kKeys - 1) / kKeys;
+    // this CTA's key tiles: a contiguous share of the row's (a CTA with none still sends an end record)
+    const int per_split = (ntiles + a.splits - 1) / a.splits;
+    const int t_lo = min(ntiles, split * per_split), t_hi = min(ntiles, t_lo + per_split);
 
     if (warp == 2) {
         // ============================== key decoder ==============================
         uint32_t rk = 0, rph = 0;
         const int mp = c.max_pages_per_row;
-        for (int t = 0; t < ntiles; ++t) {
-            const int k0 = t * kKeys, nk = min(kKeys, n - k0);
+        const int64_t ms = c.max_slots;
+        // The raw loads of a key tile (its 8 block-table entries and 128 slot positions, indexes clamped into
+        // the row) are issued one tile ahead, so their latency hides behind the previous tile's record.
+        struct Raw {
+            int page, kp[4];
+        };
+        auto load_raw = [&](int t, Raw &r) {
+            r.page = c.block_table[(int64_t)row * mp + min(t * kPages + (lane & (kPages - 1)), mp - 1)];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r.kp[i] = c.slot_pos[(int64_t)row * ms + min((int64_t)t * kKeys + i * 32 + lane, ms - 1)];
+        };
+        const int t_end = max(t_hi, t_lo + 1);
+        Raw cur, nxt;
+        if (t_lo < t_hi) load_raw(t_lo, cur);
+        for (int t = t_lo; t < t_end; ++t) {
+            if (t > t_lo) cur = nxt;
+            if (t + 1 < t_hi) load_raw(t + 1, nxt);
+            const bool none = t >= t_hi;           // the end record of a CTA without key tiles
+            const int k0 = t * kKeys, nk = none ? 0 : min(kKeys, n - k0);
             int page = -1;
             bool ok = false;
-            if (lane < kPages && k0 + lane * 16 < n) {
-                page = c.block_table[(int64_t)row * mp + min(t * kPages + lane, mp - 1)];
+            if (!none && lane < kPages && k0 + lane * 16 < n) {
+                page = cur.page;
                 ok = page >= 0 && page < c.num_pages;
                 if (!ok && qt == 0) report(a.status, KVC_DEV_BAD_PAGE, row);
             }
@@ -187,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 4; ++i) {
                 const int key = i * 32 + lane;
                 const bool v = key < nk && ((okmask >> (key >> 4)) & 1u);
-                kp[i] = v ? c.slot_pos[(int64_t)row * c.max_slots + k0 + key] : INT32_MAX;
+                kp[i] = v ? cur.kp[i] : INT32_MAX;
                 if (v) {
                     kmin = min(kmin, kp[i]);
                     kmax = max(kmax, kp[i]);
@@ -198,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
                 kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
             }
-            const bool last = t == ntiles - 1;
+            const bool last = t == max(t_hi, t_lo + 1) - 1;
             if (kmin > qlast && !last) continue;   // no column of this CTA sees any key of the tile
             if (!wait_bar(&ctl.r_empty[rk], rph ^ 1, ctl, a.status, row)) break;
             KeyRec &R = rec[rk];
@@ -365,13 +394,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 S = s * ex2(m - M);
                 for (int u = 0; u < 3; ++u) S += ctl.part_s[u][col] * ex2(ctl.part_m[u][col] - M);
             }
-            a.q.lse[((int64_t)(seq * c.num_layers + layer) * a.q.num_q_heads + kvh * G + g) * a.q.max_q + j] =
-                S > 0.f ? (M + __log2f(S)) * 0.6931471805599453f : -INFINITY;
+            if (a.splits == 1)
+                a.q.lse[((int64_t)(seq * c.num_layers + layer) * a.q.num_q_heads + kvh * G + g) * a.q.max_q + j] =
+                    S > 0.f ? (M + __log2f(S)) * 0.6931471805599453f : -INFINITY;
+            ctl.fin_m[col] = M;
+            ctl.fin_s[col] = S;
         }
     }
     if (*(volatile int32_t *)&ctl.abort) {
         const uint64_t t0 = now_ns();
         while (now_ns() - t0 < 50000ull) {}
+    }
+    if (a.splits > 1) {
+        // the cluster's CTAs split the row's keys: CTA 0 merges their (max, sum) per column through distributed
+        // shared memory; the closing cluster barrier keeps every CTA's shared memory alive until then
+        cg::cluster_group cl = cg::this_cluster();
+        cl.sync();
+        if (split == 0 && threadIdx.x < nqt * G) {
+            const int col = threadIdx.x, j = j0 + col / G, g = col % G;
+            if (j < nq) {
+                float M = -INFINITY;
+                for (int r = 0; r < a.splits; ++r) M = fmaxf(M, cl.map_shared_rank(&ctl, r)->fin_m[col]);
+                float S = 0.f;
+                if (M != -INFINITY)
+                    for (int r = 0; r < a.splits; ++r) {
+                        const Ctrl *p = cl.map_shared_rank(&ctl, r);
+                        S += p->fin_s[col] * ex2(p->fin_m[col] - M);
+                    }
+                a.q.lse[((int64_t)(seq * c.num_layers + layer) * a.q.num_q_heads + kvh * G + g) * a.q.max_q + j] =
+                    S > 0.f ? (M + __log2f(S)) * 0.6931471805599453f : -INFINITY;
+            }
+        }
+        cl.sync();
     }
     tc_fence_before();
     __syncthreads();
@@ -432,10 +486,36 @@ cudaError_t launch_lse_tc_t(const CacheView &c, const QueryView &q, int32_t *sta
     static int smem_set[kMaxDevices];
     cudaError_t e = dyn_smem_at_least((const void *)lse_tc_kernel<D>, PL::kBytes, smem_set);
     if (e != cudaSuccess) return e;
-    const int64_t grid = (int64_t)c.rows * args.tiles_q;
-    if (grid <= 0) return cudaSuccess;
-    lse_tc_kernel<D><<<(unsigned)grid, kThreads, PL::kBytes, stream>>>(tk, tq, args);
-    return cudaGetLastError();
+    const int64_t units = (int64_t)c.rows * args.tiles_q;
+    if (units <= 0) return cudaSuccess;
+    // One CTA per SM: split each column tile's keys over the cluster size S (1..8) that minimises the waves of
+    // CTAs per unit of work, ceil(units * S / SMs) / S, keeping at least four key tiles per CTA.
+    const int sms = device_sms();
+    const int64_t ntiles = (c.max_slots + kKeys - 1) / kKeys;
+    int S = 1;
+    double best = (double)((units + sms - 1) / sms);
+    for (int t = 2; t <= 8; ++t) {
+        if (ntiles < 4 * t) break;
+        const double cost = (double)((units * t + sms - 1) / sms) / t;
+        if (cost < best - 1e-9) {
+            best = cost;
+            S = t;
+        }
+    }
+    args.splits = S;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * S));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = PL::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, lse_tc_kernel<D>, tk, tq, args);
 }
 
 }  // namespace
