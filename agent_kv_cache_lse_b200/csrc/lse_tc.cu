@@ -351,22 +351,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int32_t *kp = R.kpos + kq * 32;
                 tmem_wait32(r);
                 float lm = -INFINITY;
+                if (__all_sync(0xffffffffu, all)) {
+                    // no column of the warp needs the mask (decided per warp, so the masked path below costs the
+                    // fast one nothing); the scaling runs as packed f32x2 products
+                    const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    float x = __uint_as_float(r[u]) * sc;
-                    if (!all) {
+                    for (int u = 0; u < 32; u += 2) {
+                        const float2 x = __fmul2_rn(make_float2(__uint_as_float(r[u]), __uint_as_float(r[u + 1])), sc2);
+                        r[u] = __float_as_uint(x.x);
+                        r[u + 1] = __float_as_uint(x.y);
+                        lm = fmaxf(lm, fmaxf(x.x, x.y));
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        float x = __uint_as_float(r[u]) * sc;
                         const int p = kp[u];   // absent or unreadable keys hold INT32_MAX and are never visible
                         if (p > qpos || p == INT32_MAX) x = -INFINITY;
+                        r[u] = __float_as_uint(x);
+                        lm = fmaxf(lm, x);
                     }
-                    r[u] = __float_as_uint(x);
-                    lm = fmaxf(lm, x);
                 }
                 if (lm != -INFINITY) {
                     const float nm = fmaxf(m, lm);
-                    float add = 0.f;
+                    const float2 nm2 = make_float2(-nm, -nm);
+                    float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) add += ex2(__uint_as_float(r[u]) - nm);
-                    s = s * ex2(m - nm) + add;
+                    for (int u = 0; u < 32; u += 2) {
+                        const float2 d = __fadd2_rn(make_float2(__uint_as_float(r[u]), __uint_as_float(r[u + 1])), nm2);
+                        acc = __fadd2_rn(acc, make_float2(ex2(d.x), ex2(d.y)));
+                    }
+                    s = s * ex2(m - nm) + (acc.x + acc.y);
                     m = nm;
                 }
             }
