@@ -16,7 +16,9 @@
 namespace kvc {
 namespace {
 
-__global__ void __launch_bounds__(kRowThreads, 1) lrfu_kernel(LrfuArgs a) {
+// At most 96 registers (512 x 96 of the SM's 65,536): the round runs the ratchet's confidence CTAs beside this
+// kernel, and the spare registers let two of them share each SM that holds an LRFU CTA.
+__global__ void __maxnreg__(96) lrfu_kernel(LrfuArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RowCtx rc = row_ctx();
     lrfu_row(a, rc, smem_raw);
