@@ -338,24 +338,36 @@ struct UpdArgs {
     int32_t *budget;
     int32_t num_seqs, steps, hist_len;
     kvc_ratchet_params p;
+    int32_t staged;     // the call's history (window - 1 + steps floats per warp) fits shared memory
 };
 
 // One warp per sequence: the lanes share each window's minimum and the history shift; lane 0 keeps
-// the least-squares sums and takes the decision.
+// the least-squares sums and takes the decision.  The warp first copies the sequence's history into shared
+// memory with all its loads in flight, so the windows' minima read shared memory instead of waiting on a
+// global load per window (calls whose history does not fit read global memory).
 __global__ void ratchet_update_kernel(UpdArgs a) {
+    extern __shared__ float hs_all[];   // [warps of the CTA][window - 1 + steps]
     const int lane = threadIdx.x & 31;
     const int seq = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (seq >= a.num_seqs) return;
     kvc_ratchet_seq_state s = a.st[seq];
     float *h = a.hist + (int64_t)seq * a.hist_len;
     const int W = a.p.window, R = a.p.stride;
+    const int nh = W - 1 + a.steps;     // the entries this call reads
+    const float *hs = h;
+    if (a.staged) {
+        float *st = hs_all + (size_t)(threadIdx.x >> 5) * nh;
+        for (int k = lane; k < nh; k += 32) st[k] = h[k];
+        __syncwarp();
+        hs = st;
+    }
     const int64_t t0 = s.steps_seen, t1 = t0 + a.steps;
     const int64_t base = t0 - (W - 1);  // global step held by h[0]
     int64_t j = s.next_window;
     for (; (int64_t)R * j + W <= t1; ++j) {
         const int64_t ws = (int64_t)R * j;
         float y = INFINITY;
-        for (int64_t t = ws + lane; t < ws + W; t += 32) y = fminf(y, h[t - base]);
+        for (int64_t t = ws + lane; t < ws + W; t += 32) y = fminf(y, hs[t - base]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) y = fminf(y, __shfl_xor_sync(0xffffffffu, y, o));
         if (ws >= s.last_expand_step) {
@@ -386,7 +398,7 @@ __global__ void ratchet_update_kernel(UpdArgs a) {
     // reads before it writes, so the overlapping forward copy is safe
     for (int k0 = 0; k0 < W - 1; k0 += 32) {
         const int k = k0 + lane;
-        const float v = k < W - 1 ? h[k + a.steps] : 0.f;
+        const float v = k < W - 1 ? hs[k + a.steps] : 0.f;
         __syncwarp();
         if (k < W - 1) h[k] = v;
         __syncwarp();
@@ -463,7 +475,9 @@ cudaError_t launch_ratchet(const float *logits, int32_t num_seqs, int32_t steps,
         if (e != cudaSuccess) return e;
     }
     UpdArgs u{st, hist, budget, num_seqs, steps, l.hist_len, p};
-    ratchet_update_kernel<<<(num_seqs + 3) / 4, 128, 0, stream>>>(u);
+    const size_t upd_smem = (size_t)4 * (p.window - 1 + steps) * sizeof(float);
+    u.staged = upd_smem <= 48 * 1024;
+    ratchet_update_kernel<<<(num_seqs + 3) / 4, 128, u.staged ? upd_smem : 0, stream>>>(u);
     return cudaGetLastError();
 }
 
