@@ -604,12 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (lane < 8) {
-                uint32_t w = 0;
-                for (int bit = 0; bit < 32; ++bit) {
-                    const int key = lane * 32 + bit;
-                    if (key < n_keys && ((okmask >> (key >> 4)) & 1u)) w |= 1u << bit;
-                }
-                ctl.kvstage[parity][lane] = w;
+                // readable keys lane*32 .. lane*32+31: below n_keys, in one of the lane's two pages that loaded
+                const int k0l = lane * 32;
+                const uint32_t keym =
+                    n_keys >= k0l + 32 ? 0xFFFFFFFFu : (n_keys <= k0l ? 0u : ((1u << (n_keys - k0l)) - 1u));
+                const uint32_t pg = (okmask >> (2 * lane)) & 3u;
+                const uint32_t pagem = ((pg & 1u) ? 0x0000FFFFu : 0u) | ((pg & 2u) ? 0xFFFF0000u : 0u);
+                ctl.kvstage[parity][lane] = keym & pagem;
             }
             const int layer = (int)(rr / c.num_kv_heads), kvh = (int)(rr % c.num_kv_heads);
             if (lane == 0) {
