@@ -74,7 +74,8 @@ def attention_lse(q: np.ndarray, k: np.ndarray, q_pos: np.ndarray, k_pos: np.nda
         mx = l.max(axis=2, initial=-np.inf)
         safe = np.where(np.isfinite(mx), mx, 0.0)
         ssum = np.exp(l - safe[:, :, None]).sum(axis=2)
-        out[:, a:b] = np.where(np.isfinite(mx), safe + np.log(ssum), -np.inf)
+        with np.errstate(divide="ignore"):   # log(0) of a column that sees no key; np.where takes -inf there
+            out[:, a:b] = np.where(np.isfinite(mx), safe + np.log(ssum), -np.inf)
     return out
 
 
