@@ -12,7 +12,7 @@
 // it (kNoAllocMaxRows + 1 int64 values, 128 KiB) until the process exits.  Host code
 // cannot use the array's name as a device address, so the first call on each device
 // looks the address up with cudaGetSymbolAddress (with that device current) and caches
-// it; that first call should therefore happen before any stream capture.  All calls
+// it.  All calls
 // share the array: calls whose kernels overlap on the GPU (for instance on two streams)
 // race on it and must be serialised by the caller.  Nothing in it needs to start at
 // zero: the offset kernel writes every entry it later reads.

@@ -293,7 +293,7 @@ kvc_status kvc_compact_pages(const kvc_cache *cache, const int32_t *move_src, co
  * the workspace is a fixed array inside the library (KVC_NOALLOC_MAX_ROWS + 1 int64 per
  * GPU, held from library load to process exit).  Calls for more than KVC_NOALLOC_MAX_ROWS
  * rows return KVC_ERR_UNSUPPORTED.  The first call on each device looks up the array's
- * device address (make it before any stream capture).  All calls share the array, so calls
+ * device address (a synchronous runtime query).  All calls share the array, so calls
  * whose kernels can overlap on the GPU race and must be serialised by the caller.
  */
 #define KVC_NOALLOC_MAX_ROWS 16384
