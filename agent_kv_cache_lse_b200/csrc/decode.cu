@@ -26,6 +26,13 @@
 //     every CTA adds sum_g 2^(l - M_g) / S_g to its slots' scores from the logits it kept.
 // Every sum runs in a fixed order, so results repeat bit for bit from run to run.  The kernel has
 // no spin-waits: cp.async groups always complete, and the cluster barriers are taken by all CTAs.
+//
+// Where the lanes' logits are reduce-scattered (two lanes per key) and the slot positions and scores
+// can be copied 16 bytes at a time, the kept logits leave shared memory for tensor memory (TMEM, which
+// this kernel has no other use for): each lane stores its logits of a chunk into its own TMEM lane
+// (tcgen05.st), and each chunk's stage also carries the chunk's slot positions and, when accumulating,
+// its old scores (stored to TMEM beside the logits).  Shared memory then holds only the K/V stages, so
+// every warp keeps two chunks in flight instead of one, and the final scores need no global reads.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -46,7 +53,8 @@ constexpr int kMaxGroup = 8;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxD = 128;
 constexpr int kMaxRing = 4;                 // stages per warp
-constexpr size_t kSmemLimit = 220 * 1024;   // dynamic bytes per CTA
+constexpr int kTmRing = 3;                  // stages per warp with the logits in TMEM
+constexpr int kTmMinCluster = 1;            // smallest cluster of the TMEM plan
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct DecodeArgs {
@@ -72,7 +80,13 @@ struct DecodeShared {
     float M[kMaxGroup], S[kMaxGroup];
     float pw[kWarps][16 * kMaxGroup];                    // per-warp probabilities of a chunk [key][head]
     int32_t bad;
+    uint32_t tmem;                                       // TMEM base address (logits kept in TMEM)
 };
+
+// dynamic shared memory per CTA: 227 KiB per block less 9 KiB for the static part (rounded up to 128 bytes)
+static_assert(sizeof(DecodeShared) + 128 <= 9 * 1024, "static shared memory");
+constexpr size_t kSmemLimit = (227 - 9) * 1024;
+constexpr size_t kSmemLimitTm = kSmemLimit;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -102,6 +116,58 @@ __device__ __forceinline__ void lds8(const float *p, float2 (&x)[4]) {
     x[3] = make_float2(b.z, b.w);
 }
 
+// tensor-memory stores and loads of one warp's 32 lanes (32x32b shape: thread t owns TMEM lane base + t)
+__device__ __forceinline__ void tm_st(uint32_t taddr, const float (&v)[1]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v[0])) : "memory");
+}
+__device__ __forceinline__ void tm_st(uint32_t taddr, const float (&v)[2]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(__float_as_uint(v[0])),
+                 "r"(__float_as_uint(v[1])) : "memory");
+}
+__device__ __forceinline__ void tm_st(uint32_t taddr, const float (&v)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3])) : "memory");
+}
+__device__ __forceinline__ void tm_ld8(uint32_t taddr, uint32_t *r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr) : "memory");
+}
+// after tcgen05.wait::ld: ties the loaded registers to a point after the wait
+__device__ __forceinline__ void tm_hold8(uint32_t *r) {
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+}
+
+// warp-level tensor-core steps of the bf16 path (one 16-key chunk per warp; see decode_kernel)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+// c += A (16 x 16, row) * B (16 x 8, col), bf16 operands, fp32 accumulate
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// (x, y) -> bf16x2 with x in the low half, and the rounding remainders as a second bf16x2
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x - __low2float(h), y - __high2float(h));
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -111,13 +177,23 @@ __device__ __forceinline__ float ex2(float x) {
 // 2^(x - ref): zero for x = -inf (an empty max or a masked logit), whatever ref is; ref is finite otherwise
 __device__ __forceinline__ float weight(float x, float ref) { return x == -INFINITY ? 0.f : ex2(x - ref); }
 
-template <typename T, int D, int GM, int RW>
+template <typename T, int D, int GM, int RW, bool TM, bool MM>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     constexpr int LK = D / 8;        // lanes per key
     constexpr int KW = 32 / LK;      // keys per warp step
     constexpr int MAXSTEPS = 16 / KW;
     // reduce-scatter of the dot products when every lane can end with whole ones and the partials fit
     constexpr bool kRS = MAXSTEPS * GM >= LK && MAXSTEPS * GM <= 32;
+    static_assert(!TM || (kRS && LK == 2 * MAXSTEPS), "TMEM logits need the reduce-scatter with two lanes per key");
+    // TMEM logits: a lane keeps RL logits per chunk (two lanes per key), in columns [i * RL, i * RL + RL) of
+    // its warp's 256; the old scores sit in columns kTmCap * RL + i
+    constexpr int RL = kRS ? MAXSTEPS * GM / LK : 1;
+    constexpr int kTmCap = (256 / (RL + 1)) / 8 * 8;  // chunks per warp the columns hold (a multiple of 8)
+    // MM: the chunk's two contractions on the tensor cores (bf16, four-head groups, 16-slot chunks, logits in TMEM)
+    static_assert(!MM || (TM && GM == 4 && sizeof(T) == 2 && RL == 2), "tensor-core chunks: bf16, G' = 4, TMEM");
+    constexpr int RB = D * (int)sizeof(T);  // bytes of a key's row
+    constexpr int NS = D / 16;              // k-steps of q . k, 16-row tiles of the output
+    constexpr float kSlack = 8.f;           // MM: the running maximum moves only when a logit passes it by 8 (log2)
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ DecodeShared sh;
     cg::cluster_group cl = cg::this_cluster();
@@ -128,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int seq = row / (c.num_layers * Hkv), layer = (row / Hkv) % c.num_layers, kvh = row % Hkv;
     const uint32_t half = (uint32_t)CH * D * sizeof(T);   // bytes of a chunk's K (or V)
-    const uint32_t stage_bytes = 2 * half;
+    // a stage: the chunk's K and V rows, then (TMEM logits) its CH slot positions and CH old scores
+    const uint32_t stage_bytes = TM ? 2 * half + 8 * (uint32_t)CH : 2 * half;
     unsigned char *ring = smem + (size_t)warp * RW * stage_bytes;                      // this warp's stages
     float *lg = reinterpret_cast<float *>(smem + (size_t)kWarps * RW * stage_bytes);   // [GM][slice_cap]
     int32_t *ps = reinterpret_cast<int32_t *>(lg + (size_t)GM * a.slice_cap);          // [slice_cap] positions
@@ -149,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const T *vp = static_cast<const T *>(c.v_pool);
     const int ni = nch > warp ? (nch - warp + kWarps - 1) / kWarps : 0;  // this warp's chunks
     if (tid == 0) sh.bad = 0;
+    const bool acc_old = TM && a.scores != nullptr && a.accumulate;
 
     // page ids of this warp's chunks, 32 at a time (one per lane): batch b sits in pb[b & 1], and batch b + 1 is
     // loaded when the first chunk of batch b is issued
@@ -162,17 +240,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             const int s = i % RW;
             const bool ok = pg >= 0 && pg < c.num_pages;
             okmask = ok ? (okmask | (1u << s)) : (okmask & ~(1u << s));
+            const uint32_t dst = smem_u32(ring + (size_t)s * stage_bytes);
             if (ok) {
                 const int64_t off = ((int64_t)pg * P + (lo + (warp + i * kWarps) * CH) % P) * D;
                 const char *ks = reinterpret_cast<const char *>(kp + off);
                 const char *vs = reinterpret_cast<const char *>(vp + off);
-                const uint32_t dst = smem_u32(ring + (size_t)s * stage_bytes);
                 for (uint32_t b = lane * 16; b < half; b += 512) {
-                    cp16(dst + b, ks + b);
-                    cp16(dst + half + b, vs + b);
+                    // MM: 16-byte piece c of key row r lands at piece c ^ (r & 7), so that the eight rows an
+                    // ldmatrix phase reads fall in distinct bank groups
+                    const uint32_t db = MM ? (b & ~(uint32_t)(RB - 1)) |
+                                                 ((((b & (RB - 1)) >> 4) ^ ((b / RB) & 7)) << 4)
+                                           : b;
+                    cp16(dst + db, ks + b);
+                    cp16(dst + half + db, vs + b);
                 }
             } else {
                 bad = true;
+            }
+            if constexpr (TM) {
+                // the chunk's slot positions and old scores, 16 bytes a lane (CH is a multiple of 4 and divides
+                // max_slots, so a whole chunk lies inside the row)
+                const int64_t cs = (int64_t)row * c.max_slots + lo + (warp + i * kWarps) * CH;
+                const int nq = CH / 4;
+                if (lane < nq) cp16(dst + 2 * half + lane * 16, c.slot_pos + cs + lane * 4);
+                else if (acc_old && lane >= 16 && lane < 16 + nq)
+                    cp16(dst + 2 * half + CH * 4 + (lane - 16) * 16, a.scores + cs + (lane - 16) * 4);
             }
         }
         cp_commit();  // one group per issue, empty or not, so that the group count stays in step
@@ -183,7 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     // the slice's slot positions and the group's query slice
     const int kslot = lane / LK, sub = lane % LK;
     const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots + lo;
-    for (int i = tid; i < cnt; i += kThreads) ps[i] = pos[i];
+    if constexpr (!TM)
+        for (int i = tid; i < cnt; i += kThreads) ps[i] = pos[i];
     float2 qv[GM][4];
     {
         const T *qg = static_cast<const T *>(a.q) + hbase * D + sub * 8;
@@ -201,7 +294,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
         }
     }
+    if constexpr (TM) {
+        if (warp == 0) {  // one CTA per SM (its shared memory), so all 512 columns are free
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh.tmem)),
+                         "r"(512) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    }
     __syncthreads();
+    uint32_t tmw = 0;  // this warp's TMEM columns: lane quadrant warp % 4, column half warp / 4
+    if constexpr (TM) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        tmw = sh.tmem + (((uint32_t)(warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * 256;
+    }
 
     float m[GM], s[GM];
     float2 o[GM][4];
@@ -211,6 +317,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         s[g] = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t) o[g][t] = make_float2(0.f, 0.f);
+    }
+    // MM state.  A lane holds the heads hm = 2 (lane % 4), hm + 1: their running maxima and sums, and the output
+    // tile entries O[d][h] for d = 16 j + lane / 4 (+ 8), h = hm, hm + 1 (the mma accumulator layout); the query
+    // slice as the mma B fragments, Q[lane / 4][16 t + 2 (lane % 4) + (0, 1, 8, 9)]
+    float mm[2] = {-INFINITY, -INFINITY}, ms[2] = {0.f, 0.f};
+    float oc[MM ? NS : 1][4];
+    uint32_t qb[MM ? NS : 1][2];
+    if constexpr (MM) {
+        const int hq = lane >> 2;
+        const uint32_t *qg = reinterpret_cast<const uint32_t *>(static_cast<const T *>(a.q) + (hbase + hq) * D);
+#pragma unroll
+        for (int t = 0; t < NS; ++t) {
+            qb[t][0] = hq < G ? qg[8 * t + (lane & 3)] : 0u;
+            qb[t][1] = hq < G ? qg[8 * t + 4 + (lane & 3)] : 0u;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) oc[t][u] = 0.f;
+        }
     }
     const int steps = (CH + KW - 1) / KW;
     for (int i = 0; i < ni; ++i) {
@@ -227,8 +350,96 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         const bool page_ok = (okmask >> st) & 1u;
         const T *Ks = reinterpret_cast<const T *>(ring + (size_t)st * stage_bytes);
         const T *Vs = Ks + CH * D;
+        const int32_t *psS = reinterpret_cast<const int32_t *>(ring + (size_t)st * stage_bytes + 2 * half);
         const int il0 = (warp + i * kWarps) * CH;
-        if constexpr (kRS) {
+        if constexpr (MM) {
+            const uint32_t kb = smem_u32(Ks), vb = smem_u32(Vs);
+            if (!page_ok || il0 + 16 > cnt) {  // V rows no key may use are zeroed: P is 0 there, and 0 * NaN is not
+                for (int e = lane; e < 16 * RB / 16; e += 32) {
+                    const int key = e / (RB / 16);
+                    if (!page_ok || il0 + key >= cnt)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + e * 16), "r"(0u) : "memory");
+                }
+                __syncwarp();
+            }
+            // S[key][head] = K (16 keys x D) . Q^T: ldmatrix phase q reads keys (lane & 7) + 8 (q & 1), D piece 2t + q / 2
+            float sc4[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t rowa = kb + key * RB;
+#pragma unroll
+                for (int t = 0; t < NS; ++t) {
+                    uint32_t af[4];
+                    ldsm_x4(rowa + ((((uint32_t)(2 * t + (lane >> 4))) ^ (key & 7)) << 4), af);
+                    mma16816(sc4, af, qb[t][0], qb[t][1]);
+                }
+            }
+            // lane: keys ka = lane / 4 and ka + 8, heads hm, hm + 1; base-2 logits, hidden keys -inf
+            const int ka = lane >> 2;
+            const bool va = page_ok && il0 + ka < cnt && psS[ka] <= qpos;
+            const bool vb8 = page_ok && il0 + ka + 8 < cnt && psS[ka + 8] <= qpos;
+            const float l00 = va ? sc4[0] * a.scale_log2 : -INFINITY, l01 = va ? sc4[1] * a.scale_log2 : -INFINITY;
+            const float l10 = vb8 ? sc4[2] * a.scale_log2 : -INFINITY, l11 = vb8 ? sc4[3] * a.scale_log2 : -INFINITY;
+            float lm0 = fmaxf(l00, l10), lm1 = fmaxf(l01, l11);
+            if (__any_sync(0xffffffffu, lm0 > mm[0] + kSlack || lm1 > mm[1] + kSlack)) {
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    lm0 = fmaxf(lm0, __shfl_xor_sync(0xffffffffu, lm0, off));
+                    lm1 = fmaxf(lm1, __shfl_xor_sync(0xffffffffu, lm1, off));
+                }
+                const float n0 = fmaxf(mm[0], lm0), n1 = fmaxf(mm[1], lm1);
+                const float f0 = weight(mm[0], n0), f1 = weight(mm[1], n1);
+                ms[0] *= f0;
+                ms[1] *= f1;
+#pragma unroll
+                for (int t = 0; t < NS; ++t) {
+                    oc[t][0] *= f0;
+                    oc[t][1] *= f1;
+                    oc[t][2] *= f0;
+                    oc[t][3] *= f1;
+                }
+                mm[0] = n0;
+                mm[1] = n1;
+            }
+            const float p00 = weight(l00, mm[0]), p01 = weight(l01, mm[1]);
+            const float p10 = weight(l10, mm[0]), p11 = weight(l11, mm[1]);
+            ms[0] += p00 + p10;
+            ms[1] += p01 + p11;
+            if constexpr (TM) {
+                if (a.scores) {  // logits of key ka (+ 8 on lanes with bit 1 set, taken from lane ^ 2), old score
+                    const bool up = (lane & 2) != 0;
+                    const float x0 = __shfl_xor_sync(0xffffffffu, l10, 2), x1 = __shfl_xor_sync(0xffffffffu, l11, 2);
+                    const float lv[2] = {up ? x0 : l00, up ? x1 : l01};
+                    tm_st(tmw + (uint32_t)(i * 2), lv);
+                    if (acc_old) {
+                        const float ov[1] = {reinterpret_cast<const float *>(psS + CH)[ka + (up ? 8 : 0)]};
+                        tm_st(tmw + (uint32_t)(kTmCap * 2 + i), ov);
+                    }
+                }
+            }
+            // P as the B operand [key][head]: bf16 hi + lo (so that P keeps 16 bits of mantissa), transposed from
+            // the [key][head] rows this lane holds into the [head][key] columns the fragment wants
+            uint32_t h0, g0, h1, g1;
+            split_bf16(p00, p01, h0, g0);
+            split_bf16(p10, p11, h1, g1);
+            h0 = movm_t(h0);
+            g0 = movm_t(g0);
+            h1 = movm_t(h1);
+            g1 = movm_t(g1);
+            // O^T[d][head] += V^T (d x 16 keys) . P: ldmatrix.trans phase q reads keys (lane & 7) + 8 (q / 2),
+            // D piece 2t + (q & 1)
+            {
+                const int key = (lane & 7) + ((lane >> 4) & 1) * 8;
+                const uint32_t rowa = vb + key * RB;
+#pragma unroll
+                for (int t = 0; t < NS; ++t) {
+                    uint32_t af[4];
+                    ldsm_x4_t(rowa + ((((uint32_t)(2 * t + ((lane >> 3) & 1))) ^ (key & 7)) << 4), af);
+                    mma16816(oc[t], af, h0, h1);
+                    mma16816(oc[t], af, g0, g1);
+                }
+            }
+        } else if constexpr (kRS) {
             // the chunk's V = MAXSTEPS * GM partial dots per lane, reduced over the key's LK lanes by halving:
             // lane sub ends with the R complete dots v = sub * R + r (step v / GM, head v % GM)
             constexpr int V = MAXSTEPS * GM, R = V / LK;
@@ -237,7 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
 #pragma unroll
             for (int t = 0; t < MAXSTEPS; ++t) {
                 const int kk = t * KW + kslot;
-                const bool v = t < steps && page_ok && kk < CH && il0 + kk < cnt && ps[il0 + kk] <= qpos;
+                const bool v = t < steps && page_ok && kk < CH && il0 + kk < cnt &&
+                               (TM ? psS[kk] : ps[il0 + kk]) <= qpos;
                 vis |= (v ? 1u : 0u) << t;
                 float2 x[4];
                 if (v) lds8(Ks + kk * D + sub * 8, x);
@@ -273,10 +485,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             for (int r = 0; r < R; ++r) {
                 const int v = vbase + r, t = v / GM, g = v % GM, kk = t * KW + kslot;
                 lv[r] = ((vis >> t) & 1u) ? d[r] * a.scale_log2 : -INFINITY;
-                if (g < G && t < steps && kk < CH && il0 + kk < cnt) lg[(size_t)g * a.slice_cap + il0 + kk] = lv[r];
+                if (!TM && g < G && t < steps && kk < CH && il0 + kk < cnt) lg[(size_t)g * a.slice_cap + il0 + kk] = lv[r];
 #pragma unroll
                 for (int h = 0; h < GM; ++h)
                     if (h == g) cm[h] = fmaxf(cm[h], lv[r]);
+            }
+            if constexpr (TM) {
+                if (a.scores) {  // the lane's logits of chunk i, and the old score of the key its lane pair sums
+                    tm_st(tmw + (uint32_t)(i * R), lv);
+                    if (acc_old) {
+                        const int ko = (sub >> 1) * KW + kslot;
+                        const float ov[1] = {ko < CH ? reinterpret_cast<const float *>(psS + CH)[ko] : 0.f};
+                        tm_st(tmw + (uint32_t)(kTmCap * R + i), ov);
+                    }
+                }
             }
 #pragma unroll
             for (int g = 0; g < GM; ++g) {
@@ -396,10 +618,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         __syncwarp();  // every lane is done with stage st before the next issue refills it
     }
     cp_wait<0>();
+    if constexpr (MM) {  // the sums over the lanes that share heads; the maxima already agree across them
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            ms[0] += __shfl_xor_sync(0xffffffffu, ms[0], off);
+            ms[1] += __shfl_xor_sync(0xffffffffu, ms[1], off);
+        }
+        if (lane < GM / 2) {
+            sh.wm[warp][2 * lane] = mm[0];
+            sh.wm[warp][2 * lane + 1] = mm[1];
+            sh.ws[warp][2 * lane] = ms[0];
+            sh.ws[warp][2 * lane + 1] = ms[1];
+        }
+        if (lane == 0 && bad) sh.bad = 1;
+    }
     // the warp's totals: the output over its key lanes (lanes that share sub); the sum over the lanes that
     // hold distinct probabilities (all of them after the reduce-scatter, else one lane group per key)
 #pragma unroll
-    for (int g = 0; g < GM; ++g) {
+    for (int g = 0; g < (MM ? 0 : GM); ++g) {
         if constexpr (kRS) {
 #pragma unroll
             for (int off = 1; off < LK; off <<= 1) s[g] += __shfl_xor_sync(0xffffffffu, s[g], off);
@@ -414,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
         }
     }
-    if (lane == 0) {
+    if (!MM && lane == 0) {
 #pragma unroll
         for (int g = 0; g < GM; ++g) {
             sh.wm[warp][g] = m[g];
@@ -424,7 +660,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     }
     __syncthreads();  // every warp is past its last chunk: the stages take the partial outputs
     float *wo = reinterpret_cast<float *>(smem);  // [kWarps][G][D]
-    if (kslot == 0)
+    if constexpr (MM) {
+        const int hm = 2 * (lane & 3);
+#pragma unroll
+        for (int t = 0; t < NS; ++t) {
+            const int d = 16 * t + (lane >> 2);
+            if (hm < G) {
+                wo[((size_t)warp * G + hm) * D + d] = oc[t][0];
+                wo[((size_t)warp * G + hm) * D + d + 8] = oc[t][2];
+            }
+            if (hm + 1 < G) {
+                wo[((size_t)warp * G + hm + 1) * D + d] = oc[t][1];
+                wo[((size_t)warp * G + hm + 1) * D + d + 8] = oc[t][3];
+            }
+        }
+    }
+    if (!MM && kslot == 0)
 #pragma unroll
         for (int g = 0; g < GM; ++g)
             if (g < G)
@@ -481,7 +732,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             if (bad) report(a.status, KVC_DEV_BAD_PAGE, row);
         }
     }
-    if (a.scores) {
+    if (MM && a.scores) {
+        // lane L holds key (L / 4) + 8 ((L >> 1) & 1), heads 2 (L & 1), + 1: the pair L, L ^ 1 sums the key's heads
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        const int hl = 2 * (lane & 1);
+        float inv[2], mg[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            inv[r] = (hl + r < G && sh.S[hl + r] > 0.f) ? 1.f / sh.S[hl + r] : 0.f;
+            mg[r] = sh.M[hl + r];
+        }
+        const int ko = (lane >> 2) + ((lane >> 1) & 1) * 8;
+        float *sc = a.scores + (int64_t)row * c.max_slots + lo;
+        for (int i0 = 0; i0 < ni; i0 += 8) {
+            uint32_t lr[16], orr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            tm_ld8(tmw + (uint32_t)(i0 * 2), lr);
+            tm_ld8(tmw + (uint32_t)(i0 * 2 + 8), lr + 8);
+            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * 2 + i0), orr);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            tm_hold8(lr);
+            tm_hold8(lr + 8);
+            tm_hold8(orr);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float part = 0.f;
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                    if (hl + r < G) part = fmaf(weight(__uint_as_float(lr[2 * b + r]), mg[r]), inv[r], part);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                const int il = (warp + (i0 + b) * kWarps) * CH + ko;
+                if (i0 + b < ni && (lane & 1) == 0 && il < cnt) sc[il] = __uint_as_float(orr[b]) + part;
+            }
+        }
+    }
+    if (TM && !MM && a.scores) {
+        // each lane pair adds its key's sum over the heads, from the logits and old scores kept in TMEM
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        float inv[RL], mg[RL];
+        bool use[RL];
+#pragma unroll
+        for (int r = 0; r < RL; ++r) {
+            const int g = (sub & 1) * RL + r;  // the head of this lane's r-th logit of a key
+            use[r] = g < G;
+            inv[r] = (g < G && sh.S[g] > 0.f) ? 1.f / sh.S[g] : 0.f;
+            mg[r] = sh.M[g];
+        }
+        const int ko = (sub >> 1) * KW + kslot;  // the key within a chunk
+        float *sc = a.scores + (int64_t)row * c.max_slots + lo;
+        for (int i0 = 0; i0 < ni; i0 += 8) {  // eight chunks a batch (kTmCap is a multiple of 8)
+            uint32_t lr[8 * RL], orr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int b = 0; b < RL; ++b) tm_ld8(tmw + (uint32_t)(i0 * RL + 8 * b), lr + 8 * b);
+            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * RL + i0), orr);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int b = 0; b < RL; ++b) tm_hold8(lr + 8 * b);
+            tm_hold8(orr);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float part = 0.f;
+#pragma unroll
+                for (int r = 0; r < RL; ++r)
+                    if (use[r]) part = fmaf(weight(__uint_as_float(lr[b * RL + r]), mg[r]), inv[r], part);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                const int il = (warp + (i0 + b) * kWarps) * CH + ko;
+                if (i0 + b < ni && (sub & 1) == 0 && ko < CH && il < cnt) sc[il] = __uint_as_float(orr[b]) + part;
+            }
+        }
+    }
+    if (!TM && a.scores) {
         float inv[GM], mg[GM];
 #pragma unroll
         for (int g = 0; g < GM; ++g) {
@@ -509,7 +828,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
         }
     }
+    if constexpr (TM) asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     cl.sync();  // peers may still be reading this CTA's shared memory
+    if constexpr (TM) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sh.tmem), "r"(512) : "memory");
+    }
 }
 
 int group_bound(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
@@ -517,18 +841,43 @@ int group_bound(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
 struct Plan {
     int C, CH, RW, cap;
     size_t smem;
+    bool tm;  // logits, slot positions and old scores through the stages and TMEM
+    bool mm;  // and the chunk's contractions on the tensor cores (bf16, G' = 4, 16-slot chunks)
 };
+
+// the reduce-scatter with two lanes per key (the TMEM layout) for head size D and group bound GM
+constexpr bool two_lanes_per_key(int D, int GM) {
+    const int LK = D / 8, KW = 32 / LK, MAXSTEPS = 16 / KW, V = MAXSTEPS * GM;
+    return V >= LK && V <= 32 && LK == 2 * MAXSTEPS;
+}
 
 // Cluster size, chunk, stages per warp and shared memory of a launch; C = 0 when nothing fits.  The chunk is
 // the largest divisor of the page size, at most 16 slots, whose two stages per warp fit; the cluster grows
 // (shrinking each CTA's logits buffer) until every warp has kMaxRing stages or C is 8.  At least two stages
 // per warp are needed: one landing while the other is worked on.
-Plan plan_for(const CacheView &c, int G, int sms) {
+//
+// With `aligned` (slot positions and scores 16-byte aligned) and the two-lanes-per-key reduce-scatter, the
+// TMEM plan comes first: three stages per warp, the smallest cluster whose warps' chunks fit the TMEM columns.
+// With bf16, G' = 4, 16-slot chunks and a 4-byte aligned query (`q4`), the chunks' contractions run as mma tiles.
+Plan plan_for(const CacheView &c, int G, int sms, bool aligned, bool q4) {
     const size_t elem = c.dtype == KVC_BF16 ? 2 : 4;
     const size_t partial = (size_t)kWarps * G * c.head_dim * 4;
     const int GM = group_bound(G);
     int C0 = 1;
     while (C0 < kMaxCluster && (int64_t)c.rows * C0 < sms) C0 <<= 1;
+    if (aligned && two_lanes_per_key(c.head_dim, GM)) {
+        const int RL = GM / 2, cap_w = (256 / (RL + 1)) / 8 * 8;
+        for (int CH = std::min(16, c.page_size); CH >= 4; --CH) {
+            if (c.page_size % CH || CH % 4 || c.max_slots % CH) continue;
+            const size_t stage = 2 * (size_t)CH * c.head_dim * elem + 8 * (size_t)CH;
+            const size_t smem = (size_t)kTmRing * kWarps * stage;
+            if (smem > kSmemLimitTm || smem < partial) continue;
+            const int64_t nch = (c.max_slots + CH - 1) / CH;
+            for (int C = std::max(C0, kTmMinCluster); C <= kMaxCluster; C <<= 1)
+                if (((nch + C - 1) / C + kWarps - 1) / kWarps <= cap_w)
+                    return Plan{C, CH, kTmRing, 0, smem, true, q4 && c.dtype == KVC_BF16 && GM == 4 && CH == 16};
+        }
+    }
     for (int CH = std::min(16, c.page_size); CH >= 1; --CH) {
         if (c.page_size % CH) continue;
         const size_t stage = 2 * (size_t)CH * c.head_dim * elem;
@@ -540,7 +889,7 @@ Plan plan_for(const CacheView &c, int G, int sms) {
             if (fixed >= kSmemLimit) continue;
             const int RW = (int)std::min<size_t>(kMaxRing, (kSmemLimit - fixed) / (kWarps * stage));
             if (RW < 2 || (size_t)RW * kWarps * stage < partial) continue;
-            if (RW > best.RW) best = Plan{C, CH, RW, (int)cap, (size_t)RW * kWarps * stage + fixed};
+            if (RW > best.RW) best = Plan{C, CH, RW, (int)cap, (size_t)RW * kWarps * stage + fixed, false, false};
             if (RW >= kMaxRing) break;
         }
         if (best.C) return best;
@@ -550,12 +899,12 @@ Plan plan_for(const CacheView &c, int G, int sms) {
 
 int sm_count() { return device_sms(); }
 
-template <typename T, int D, int GM, int RW>
+template <typename T, int D, int GM, int RW, bool TM, bool MM>
 cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                      float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, const Plan &p) {
     const int G = num_q_heads / c.num_kv_heads;
     static int smem_set[kMaxDevices];
-    cudaError_t e = dyn_smem_at_least((const void *)decode_kernel<T, D, GM, RW>, p.smem, smem_set);
+    cudaError_t e = dyn_smem_at_least((const void *)decode_kernel<T, D, GM, RW, TM, MM>, p.smem, smem_set);
     if (e != cudaSuccess) return e;
     DecodeArgs a{c, q, q_pos, num_q_heads, G, out, lse, scores, accumulate ? 1 : 0, p.CH, p.RW, p.cap,
                  (float)(1.4426950408889634 / std::sqrt((double)D)), status};
@@ -571,16 +920,27 @@ cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, in
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<T, D, GM, RW>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<T, D, GM, RW, TM, MM>, a);
 }
 
 template <typename T, int D, int GM>
 cudaError_t launch_r(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                      float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, const Plan &p) {
+    if constexpr (two_lanes_per_key(D, GM)) {
+        if constexpr (GM == 4 && sizeof(T) == 2) {
+            if (p.mm)
+                return launch_t<T, D, GM, kTmRing, true, true>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
+                                                               status, stream, p);
+        }
+        if (p.tm && !p.mm)
+            return launch_t<T, D, GM, kTmRing, true, false>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
+                                                            status, stream, p);
+    }
+    if (p.tm) return cudaErrorInvalidValue;
     switch (p.RW) {
-        case 2: return launch_t<T, D, GM, 2>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
-        case 3: return launch_t<T, D, GM, 3>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
-        default: return launch_t<T, D, GM, 4>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
+        case 2: return launch_t<T, D, GM, 2, false, false>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
+        case 3: return launch_t<T, D, GM, 3, false, false>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
+        default: return launch_t<T, D, GM, 4, false, false>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate, status, stream, p);
     }
 }
 
@@ -599,12 +959,15 @@ cudaError_t launch_g(const CacheView &c, const void *q, const int32_t *q_pos, in
 
 int decode_cluster(const CacheView &c, int32_t group) {
     if (group < 1 || group > kMaxGroup) return 0;
-    return plan_for(c, group, sm_count()).C;
+    return plan_for(c, group, sm_count(), false, false).C;
 }
 
 cudaError_t launch_decode(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                           float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, int) {
-    const Plan p = plan_for(c, num_q_heads / c.num_kv_heads, sm_count());
+    const bool aligned = (reinterpret_cast<uintptr_t>(c.slot_pos) & 15) == 0 &&
+                         (reinterpret_cast<uintptr_t>(scores) & 15) == 0;  // a null scores pointer is aligned
+    const Plan p = plan_for(c, num_q_heads / c.num_kv_heads, sm_count(), aligned,
+                            (reinterpret_cast<uintptr_t>(q) & 3) == 0);
     if (p.C == 0) return cudaErrorInvalidValue;
     const bool bf16 = c.dtype == KVC_BF16;
     if (c.head_dim == 64)

@@ -383,9 +383,12 @@ __device__ void row_ordered_ranks(RowCtx &rc, RowShared &sh, int lo, int hi, Amb
         if (amb(i)) out(i, rank++);
 }
 
+// CTAs per row: the largest power of two up to 8 that keeps the launch (rows x c CTAs) within one wave.  A row
+// kernel's 512 threads hold over half of an SM's registers, so one CTA runs per SM; a second wave would wait
+// for the first one's slowest row.
 __host__ inline int row_cluster_size(int rows, int sms) {
     int c = 1;
-    while (c < 8 && (int64_t)rows * c < 2 * (int64_t)sms) c <<= 1;
+    while (c < 8 && (int64_t)rows * c * 2 <= (int64_t)sms) c <<= 1;
     return c;
 }
 

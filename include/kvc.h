@@ -403,14 +403,22 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
  *          (added to with KVC_SCORE_ACCUMULATE) for slots < row_len only.
  * flags:   0 or KVC_SCORE_ACCUMULATE.
  * Limits:  num_q_heads / num_kv_heads <= 8.  Each CTA of the row's cluster (at most 8 CTAs) keeps
- *          its slice's logits and positions, (G' + 1) * 4 * ceil(max_slots / 8) bytes (G' = the
- *          group size rounded up to a power of two), beside at least two K/V stages per warp, all
- *          within 220 KiB; a stage holds a chunk of 16 slots of one page, shrinking to 8, 4, 2 or 1
- *          slots (slower) when 16 do not fit.  For bf16 and head_dim 128, 16-slot chunks serve rows
- *          up to 94,208 / 62,720 / 37,632 / 20,864 slots at G = 1 / 2 / 4 / 8, and the longest rows
- *          accepted are 217,088 / 144,720 / 83,552 / 42,768 slots; longer ones return
- *          KVC_ERR_UNSUPPORTED.  d_status reports a bad page or a bad row length; the affected
- *          row's results are then undefined.
+ *          its slice's logits until the row's LSE is known, in one of two places (G' = the group
+ *          size rounded up to a power of two):
+ *          - tensor memory, when slot_pos and scores start on 16-byte boundaries, G' is 2 or 4 at
+ *            head_dim 128 (2, 4 or 8 at head_dim 64) and the page size has a divisor that is a
+ *            multiple of 4: the stages then also carry the chunk's positions and old scores, and
+ *            every warp keeps two chunks in flight.  Rows up to 131,072 / 81,920 slots at G' = 2 / 4
+ *            (49,152 at G' = 8) with 16-slot chunks;
+ *          - otherwise shared memory: (G' + 1) * 4 * ceil(max_slots / 8) bytes of logits and
+ *            positions beside at least two K/V stages per warp, within 218 KiB; a stage holds a
+ *            chunk of 16 slots of one page, shrinking to 8, 4, 2 or 1 slots (slower) when 16 do
+ *            not fit.  For bf16 and head_dim 128, 16-slot chunks serve rows up to 92,416 / 61,568
+ *            / 36,864 / 20,480 slots at G = 1 / 2 / 4 / 8.
+ *          The longest rows accepted (the shared-memory bound, which the call checks whatever the
+ *          pointers) are 215,040 / 143,360 / 82,736 / 42,320 slots at G = 1 / 2 / 4 / 8 for bf16
+ *          and head_dim 128; longer ones return KVC_ERR_UNSUPPORTED.  d_status reports a bad page
+ *          or a bad row length; the affected row's results are then undefined.
  * Every sum runs in a fixed order: results repeat bit for bit.  One cluster of up to 8 CTAs
  * per row, exchanging maxima, sums and partial outputs through distributed shared memory.
  */

@@ -94,6 +94,8 @@ CASES = {
     "gqa7": dict(Hq=28, Hkv=4, ctx=(2100,), seed=33),
     "gqa1_f32_d64": dict(Hq=4, Hkv=4, D=64, dtype="f32", ctx=(3000,), seed=34),
     "gqa8_d64": dict(Hq=16, Hkv=2, D=64, ctx=(2500,), seed=35),
+    "gqa4_d64": dict(Hq=8, Hkv=2, D=64, ctx=(2222, 999), S=2, seed=46),
+    "gqa3": dict(Hq=24, Hkv=8, ctx=(1800,), seed=47),
     "gqa2_f32": dict(Hq=4, Hkv=2, dtype="f32", ctx=(1111,), seed=36),
     "short_rows": dict(S=2, ctx=(17, 300), seed=37),
 }
@@ -190,6 +192,49 @@ def test_decode_host_validation():
                                  torch.zeros(q9.shape[:3], device=DEV), None, 0)
 
 
+def test_decode_unaligned_scores_keep_logits_in_shared_memory():
+    """Scores that do not start on a 16-byte boundary cannot ride in the stages' 16-byte copies, so the kernel
+    keeps the logits in shared memory instead of TMEM (and forms the dot products on the FMA pipes, not the
+    tensor cores): both layouts match the oracle, and each other within the same bounds."""
+    w = H.build(spec_of(ctx=(3001,), seed=45))
+    q, q_pos = decode_inputs(w)
+    R, M = w.spec.rows, w.spec.max_slots
+    base = torch.full((R * M + 1,), -7.0, device=DEV)
+    shifted = base[1:].view(R, M)
+    assert shifted.data_ptr() % 16 != 0
+    out, lse, status = run(w, q, q_pos, shifted)
+    assert kvc.device_status(status)[0] == 0
+    check(w, q, q_pos, out, lse, shifted, range(R), "unaligned scores")
+    assert torch.all(shifted[:, 3001:] == -7.0) and base[0] == -7.0
+    aligned = torch.full((R, M), -7.0, device=DEV)
+    out2, lse2, _ = run(w, q, q_pos, aligned)
+    check(w, q, q_pos, out2, lse2, aligned, range(R), "aligned scores")
+    torch.testing.assert_close(out, out2, rtol=2e-4, atol=4e-5)
+    torch.testing.assert_close(lse, lse2, rtol=0, atol=4e-5)
+    torch.testing.assert_close(aligned, shifted, rtol=2e-3, atol=2e-6)
+
+
+def test_decode_unaligned_query_takes_the_simt_chunks():
+    """A query that does not start on a 4-byte boundary cannot feed the tensor-core chunks (their query fragments are
+    bf16 pairs): the kernel forms the dot products on the FMA pipes instead; both match the oracle."""
+    w = H.build(spec_of(S=2, ctx=(1700, 2900), seed=48))
+    q, q_pos = decode_inputs(w)
+    base = torch.empty(q.numel() + 1, dtype=q.dtype, device=DEV)
+    qs = base[1:].view(q.shape)
+    qs.copy_(q)
+    assert qs.data_ptr() % 4 != 0
+    R, M = w.spec.rows, w.spec.max_slots
+    scores = torch.full((R, M), -7.0, device=DEV)
+    out, lse, status = run(w, qs, q_pos, scores)
+    assert kvc.device_status(status)[0] == 0
+    check(w, q, q_pos, out, lse, scores, range(R), "unaligned query")
+    s2 = torch.full((R, M), -7.0, device=DEV)
+    out2, lse2, _ = run(w, q, q_pos, s2)
+    torch.testing.assert_close(out, out2, rtol=2e-4, atol=4e-5)
+    torch.testing.assert_close(lse, lse2, rtol=0, atol=4e-5)
+    torch.testing.assert_close(scores, s2, rtol=2e-3, atol=2e-6)
+
+
 def test_decode_long_row_many_chunks_per_warp():
     """A 90,000-slot row (one query head per KV head, the longest the logits buffer takes at this width): each
     warp streams about 88 chunks, so its page ids come in three batches of 32."""
@@ -219,7 +264,7 @@ def test_decode_full_size_sampled_rows():
 
 def test_decode_bench_workload_sampled_rows():
     """The workload and launch configuration bench.py --decode times: one layer of the batch of 16 sequences
-    (context 8K-33K, 128 rows, clusters of 8), checked on sampled rows."""
+    (context 8K-33K, 128 rows), checked on sampled rows."""
     spec = synth.batch16(num_layers=1)
     w = H.build(spec)
     q, q_pos = decode_inputs(w)

@@ -155,7 +155,7 @@ def test_decode_host_validation_without_gpu():
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="a supported size would launch the kernel on fake pointers")
-@pytest.mark.parametrize("group,limit", [(1, 217088), (2, 144720), (4, 83552), (8, 42768)])
+@pytest.mark.parametrize("group,limit", [(1, 215040), (2, 143360), (4, 82736), (8, 42320)])
 def test_decode_row_limit_matches_the_header(group, limit):
     """bf16, head_dim 128, 16-slot pages: the longest row the decode entry point takes, as the header states it.
     Without a GPU a supported size gets as far as the launch and fails there (KVC_ERR_CUDA); one page more is
