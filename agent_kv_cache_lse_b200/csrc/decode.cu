@@ -33,6 +33,21 @@
 // (tcgen05.st), and each chunk's stage also carries the chunk's slot positions and, when accumulating,
 // its old scores (stored to TMEM beside the logits).  Shared memory then holds only the K/V stages, so
 // every warp keeps two chunks in flight instead of one, and the final scores need no global reads.
+//
+// With bf16 K/V, four-head groups (G' = 4) and 16-slot chunks, a chunk's two contractions run on the
+// tensor cores as warp-level mma tiles (m16n8k16, fp32 accumulate) instead of per-lane FMAs:
+//   * S = K Q^T: the 16 keys are the tile's rows, D its k-steps, the group's heads (padded to 8) its
+//     columns; K comes from the stage with ldmatrix (each key row's 16-byte pieces XOR-swizzled by the
+//     row index as the copies land, so an ldmatrix phase hits eight bank groups), Q sits in registers;
+//   * the running maximum moves only when some logit passes it by more than 8 (base 2), which one warp
+//     vote decides; otherwise the chunk's probabilities 2^(l - m) (at most 2^8) are taken against the
+//     maximum as it stands.  A maximum that differs from the true one cancels in O / S and M + log2 S;
+//   * O^T += V^T P: D is the tile's rows (ldmatrix.trans of the V rows), the keys its k-steps and the
+//     heads its columns; P goes in as a bf16 high part plus a bf16 remainder (two mma per tile), so the
+//     products keep 16 bits of P's mantissa, and reaches the B-operand layout by an 8x8 register
+//     transpose (movmatrix) of the S accumulator's [key][head] pairs.
+// A lane then holds the heads 2 (lane % 4), + 1 of keys lane / 4 and lane / 4 + 8; the kept logits go to
+// TMEM two to a lane (the lanes with bit 1 set take the second key from lane ^ 2).
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
