@@ -12,8 +12,9 @@
 // The output feeds the same top-budget selection as the LRFU values.
 //
 // One CTA per row.  Rows of up to 34,816 slots keep their scores in registers (1,024 threads x 34) and
-// their step ids in shared memory, so scores and positions are read once; longer rows take three passes
-// over global memory.  Pass 1 finds max |s| of the row, which fixes a power-of-two scale; pass 2
+// their step ids in shared memory, so scores and positions are read once; a position's step comes from a
+// table of the step at every 2^sh-th position (advanced past any start inside the bucket) instead of a
+// binary search.  Longer rows take three passes over global memory.  Pass 1 finds max |s| of the row, which fixes a power-of-two scale; pass 2
 // adds every score, rounded to a 64-bit fixed-point integer at that scale, into its step's sum in
 // shared memory (integer adds, so the sums do not depend on the order of the atomics; a warp whose
 // lanes share a step adds once); pass 3 writes the blend.  The fixed point carries each score to
@@ -39,6 +40,30 @@ struct StepArgs {
     int32_t *status;
 };
 
+// Step tables up to this size get one copy of the step sums per warp: a warp's adds then never wait on
+// another warp's adds to the same step (neighbouring slots share steps, so all warps of a CTA would).
+constexpr int kPrivSteps = 64;
+
+// The exact sum over the warp of 64-bit fixed-point values |x| <= 2^39, from two 32-bit reductions:
+// x = hi * 2^20 + lo with |hi| <= 2^19 and 0 <= lo < 2^20, so neither 32-lane sum overflows.
+__device__ __forceinline__ long long warp_sum_fixed(long long x) {
+    const int hs = __reduce_add_sync(0xffffffffu, (int)(x >> 20));
+    const unsigned ls = __reduce_add_sync(0xffffffffu, (unsigned)(x & 0xFFFFF));
+    return ((long long)hs << 20) + (long long)ls;
+}
+
+// adds one warp's (sum, count) of step k: into the warp's own copy when there are copies
+__device__ __forceinline__ void add_step(int64_t *sum, int32_t *cnt, int64_t *wsum, int32_t *wcnt, int stride,
+                                         int warp, int k, long long t, int c) {
+    if (wsum) {
+        atomicAdd(reinterpret_cast<unsigned long long *>(&wsum[warp * stride + k]), (unsigned long long)t);
+        atomicAdd(&wcnt[warp * stride + k], c);
+    } else {
+        atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k]), (unsigned long long)t);
+        atomicAdd(&cnt[k], c);
+    }
+}
+
 __device__ __forceinline__ int step_of(const int32_t *starts, int ns, int32_t pos) {
     int lo = 0, hi = ns;  // the answer is in [lo, hi): starts[lo] <= pos (starts[0] = 0 <= pos for pos >= 0)
     while (hi - lo > 1) {
@@ -57,9 +82,12 @@ __global__ void __launch_bounds__(kThreads) step_scores_kernel(StepArgs a) {
     int64_t *sum = reinterpret_cast<int64_t *>(smem);                    // [max_steps]
     int32_t *cnt = reinterpret_cast<int32_t *>(sum + a.max_steps);        // [max_steps]
     int32_t *starts = cnt + a.max_steps;                                  // [max_steps]
+    const bool priv = a.max_steps <= kPrivSteps;
+    int64_t *wsum = priv ? sum + 2 * a.max_steps : nullptr;               // [warps][max_steps] per-warp copies
+    int32_t *wcnt = priv ? reinterpret_cast<int32_t *>(wsum + (kThreads / 32) * a.max_steps) : nullptr;
     __shared__ float red[kThreads / 32];
     __shared__ int bad;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const int n = c.row_len[row];
     const int ns = a.num_steps[seq];
@@ -81,6 +109,11 @@ __global__ void __launch_bounds__(kThreads) step_scores_kernel(StepArgs a) {
         cnt[k] = 0;
         if ((k == 0 && v != 0) || (k > 0 && v <= st[k - 1])) bad = 1;
     }
+    if (priv)
+        for (int e = tid; e < (kThreads / 32) * a.max_steps; e += kThreads) {
+            wsum[e] = 0;
+            wcnt[e] = 0;
+        }
     const float *s = a.scores + (int64_t)row * c.max_slots;
     const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots;
     // pass 1: max |s|
@@ -111,16 +144,10 @@ __global__ void __launch_bounds__(kThreads) step_scores_kernel(StepArgs a) {
         const unsigned vm = __ballot_sync(0xffffffffu, valid);
         const int k0 = __shfl_sync(0xffffffffu, k, __ffs(vm | 1u) - 1);
         if (vm == 0xffffffffu && __all_sync(0xffffffffu, k == k0)) {
-            long long t = qv;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-            if (lane == 0) {
-                atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k0]), (unsigned long long)t);
-                atomicAdd(&cnt[k0], 32);
-            }
+            const long long t = warp_sum_fixed(qv);
+            if (lane == 0) add_step(sum, cnt, wsum, wcnt, a.max_steps, warp, k0, t, 32);
         } else if (valid) {
-            atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k]), (unsigned long long)qv);
-            atomicAdd(&cnt[k], 1);
+            add_step(sum, cnt, wsum, wcnt, a.max_steps, warp, k, qv, 1);
         }
     }
     __syncthreads();
@@ -131,8 +158,14 @@ __global__ void __launch_bounds__(kThreads) step_scores_kernel(StepArgs a) {
     // step utilities, in place of the sums (as doubles)
     double *u = reinterpret_cast<double *>(sum);
     for (int k = tid; k < ns; k += kThreads) {
-        const long long t = sum[k];
-        u[k] = cnt[k] > 0 ? (double)t / (scale * (double)cnt[k]) : 0.0;
+        long long t = sum[k];
+        int cn = cnt[k];
+        if (priv)
+            for (int w = 0; w < kThreads / 32; ++w) {
+                t += wsum[w * a.max_steps + k];
+                cn += wcnt[w * a.max_steps + k];
+            }
+        u[k] = cn > 0 ? (double)t / (scale * (double)cn) : 0.0;
     }
     __syncthreads();
     // pass 3: the blend
@@ -158,9 +191,14 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
     int32_t *cnt = reinterpret_cast<int32_t *>(sum + a.max_steps);        // [max_steps]
     int32_t *starts = cnt + a.max_steps;                                  // [max_steps]
     uint16_t *sid = reinterpret_cast<uint16_t *>(starts + a.max_steps);  // [kRegThreads * kRegSlots] step ids
+    const bool priv = a.max_steps <= kPrivSteps;
+    // [warps][max_steps] per-warp copies of the sums and counts, after the step ids (8-byte aligned: the ids
+    // take 2 * kRegThreads * kRegSlots bytes and what precedes them 16 * max_steps)
+    int64_t *wsum = priv ? reinterpret_cast<int64_t *>(sid + kRegThreads * kRegSlots) : nullptr;
+    int32_t *wcnt = priv ? reinterpret_cast<int32_t *>(wsum + (kRegThreads / 32) * a.max_steps) : nullptr;
     __shared__ float red[kRegThreads / 32];
     __shared__ int bad;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const int n = c.row_len[row];
     const int ns = a.num_steps[seq];
@@ -182,6 +220,11 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
         cnt[k] = 0;
         if ((k == 0 && v != 0) || (k > 0 && v <= st[k - 1])) bad = 1;
     }
+    if (priv)
+        for (int e = tid; e < (kRegThreads / 32) * a.max_steps; e += kRegThreads) {
+            wsum[e] = 0;
+            wcnt[e] = 0;
+        }
     const float *s = a.scores + (int64_t)row * c.max_slots;
     const int32_t *pos = c.slot_pos + (int64_t)row * c.max_slots;
     float v[kRegSlots];
@@ -191,6 +234,15 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
         v[j] = i < n ? s[i] : 0.f;
     }
     __syncthreads();  // the step table is in place
+    // the step of every 2^sh-th position below the last start, so that a position's step is the bucket's step
+    // advanced past the (rare) starts inside the bucket
+    __shared__ uint16_t tbl[1024];
+    const int32_t last = starts[ns - 1];
+    int sh = 0;
+    while ((last >> sh) >= 1024) ++sh;
+    const int nb = (last >> sh) + 1;
+    for (int b = tid; b < nb; b += kRegThreads) tbl[b] = (uint16_t)step_of(starts, ns, b << sh);
+    __syncthreads();
     constexpr int kPart = 8;
 #pragma unroll
     for (int h = 0; h < (kRegSlots + kPart - 1) / kPart; ++h) {  // positions in parts, to stay within the registers
@@ -205,7 +257,14 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
             const int i = tid + (h * kPart + j) * kRegThreads;
             if (h * kPart + j < kRegSlots && i < n) {
                 if (p[j] < 0) bad = 1;
-                else sid[i] = (uint16_t)step_of(starts, ns, p[j]);
+                else {
+                    int k = ns - 1;
+                    if (p[j] < last) {
+                        k = tbl[p[j] >> sh];
+                        while (starts[k + 1] <= p[j]) ++k;  // k + 1 < ns: p < last = starts[ns - 1]
+                    }
+                    sid[i] = (uint16_t)k;
+                }
             }
         }
     }
@@ -230,23 +289,23 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
         const unsigned vm = __ballot_sync(0xffffffffu, in);
         const int k0 = __shfl_sync(0xffffffffu, k, 0);
         if (vm == 0xffffffffu && __all_sync(0xffffffffu, k == k0)) {
-            long long t = qv;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-            if (lane == 0) {
-                atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k0]), (unsigned long long)t);
-                atomicAdd(&cnt[k0], 32);
-            }
+            const long long t = warp_sum_fixed(qv);
+            if (lane == 0) add_step(sum, cnt, wsum, wcnt, a.max_steps, warp, k0, t, 32);
         } else if (in) {
-            atomicAdd(reinterpret_cast<unsigned long long *>(&sum[k]), (unsigned long long)qv);
-            atomicAdd(&cnt[k], 1);
+            add_step(sum, cnt, wsum, wcnt, a.max_steps, warp, k, qv, 1);
         }
     }
     __syncthreads();
     double *u = reinterpret_cast<double *>(sum);
     for (int k = tid; k < ns; k += kRegThreads) {
-        const long long t = sum[k];
-        u[k] = cnt[k] > 0 ? (double)t / (scale * (double)cnt[k]) : 0.0;
+        long long t = sum[k];
+        int cn = cnt[k];
+        if (priv)
+            for (int w = 0; w < kRegThreads / 32; ++w) {
+                t += wsum[w * a.max_steps + k];
+                cn += wcnt[w * a.max_steps + k];
+            }
+        u[k] = cn > 0 ? (double)t / (scale * (double)cn) : 0.0;
     }
     __syncthreads();
     float *o = a.out + (int64_t)row * c.max_slots;
@@ -264,7 +323,8 @@ cudaError_t launch_step_scores(const CacheView &c, const float *scores, const in
                                const int32_t *num_steps, int32_t max_steps, float beta, float *out, int32_t *status,
                                cudaStream_t stream) {
     if (c.max_slots <= (int64_t)kRegThreads * kRegSlots && max_steps <= 65536) {
-        const size_t smem = (size_t)max_steps * (8 + 4 + 4) + (size_t)kRegThreads * kRegSlots * 2;
+        const size_t smem = (size_t)max_steps * (8 + 4 + 4) + (size_t)kRegThreads * kRegSlots * 2 +
+                            (max_steps <= kPrivSteps ? (size_t)(kRegThreads / 32) * max_steps * (8 + 4) : 0);
         static int smem_set[kMaxDevices];
         cudaError_t e = dyn_smem_at_least((const void *)step_scores_reg_kernel, smem, smem_set);
         if (e != cudaSuccess) return e;
@@ -272,7 +332,8 @@ cudaError_t launch_step_scores(const CacheView &c, const float *scores, const in
             StepArgs{c, scores, step_start, num_steps, max_steps, beta, out, status});
         return cudaGetLastError();
     }
-    const size_t smem = (size_t)max_steps * (8 + 4 + 4);
+    const size_t smem = (size_t)max_steps * (8 + 4 + 4) +
+                        (max_steps <= kPrivSteps ? (size_t)(kThreads / 32) * max_steps * (8 + 4) : 0);
     if (smem > 48 * 1024) {
         static int smem_set[kMaxDevices];
         cudaError_t e = dyn_smem_at_least((const void *)step_scores_kernel, smem, smem_set);

@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def workload(ctx=(1500, 2817, 4000), L=2, Hkv=4, seed=51, permute=False, shorten=False):
+def workload(ctx=(1500, 2817, 4000), L=2, Hkv=4, seed=51, permute=False, shorten=False, pad=3):
     spec = synth.Spec(name="stepkv", seed=seed, num_seqs=len(ctx), num_layers=L, num_q_heads=Hkv, num_kv_heads=Hkv,
                       head_dim=64, dtype="f32", ctx=list(ctx), budget=256)
     lay = synth.make_layout(spec)
@@ -30,7 +30,7 @@ def workload(ctx=(1500, 2817, 4000), L=2, Hkv=4, seed=51, permute=False, shorten
         if shorten and r % 3 == 1:
             rl[r] = n // 2
     starts = [synth.step_starts(spec, s) for s in range(spec.num_seqs)]
-    ms = max(len(x) for x in starts) + 3
+    ms = max(len(x) for x in starts) + pad
     st = torch.full((spec.num_seqs, ms), 2**31 - 1, dtype=torch.int32)
     for s, x in enumerate(starts):
         st[s, :len(x)] = x
@@ -55,13 +55,18 @@ def check(spec, out, sc, pos, rl, starts, beta, what):
         assert not bad.any(), f"{what} row {r}: {int(bad.sum())} values out of tolerance, max err {err.max()}"
 
 
-@pytest.mark.parametrize("case", ["plain", "permuted_short", "beta03", "beta1", "long_rows"])
+@pytest.mark.parametrize("case", ["plain", "permuted_short", "beta03", "beta1", "long_rows", "wide_table",
+                                  "long_wide_table"])
 def test_step_scores_parity(case):
-    """Rows up to 34,816 slots run the register-resident kernel; "long_rows" (40,000 slots) the three-pass one."""
+    """Rows up to 34,816 slots run the register-resident kernel; "long_rows" (40,000 slots) the three-pass one.
+    Step tables of up to 64 columns keep one copy of the step sums per warp; the "wide" cases (90 columns) add
+    into one shared copy instead."""
     beta = {"beta03": 0.3, "beta1": 1.0}.get(case, 0.5)
-    ctx = (40000, 1200) if case == "long_rows" else (1500, 2817, 4000)
-    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=ctx, permute=case in ("permuted_short", "long_rows"),
-                                                           shorten=case == "permuted_short")
+    ctx = (40000, 1200) if case.startswith("long") else (1500, 2817, 4000)
+    spec, cache, s, st, ns, sc, pos, rl, starts = workload(ctx=ctx, permute=case in ("permuted_short", "long_rows",
+                                                                                     "long_wide_table"),
+                                                           shorten=case == "permuted_short",
+                                                           pad=90 - 25 if "wide" in case else 3)
     out = torch.full_like(s, -5.0)
     status = torch.zeros(2, dtype=torch.int32, device=DEV)
     kvc.kvc_step_scores(cache, s, st, ns, out, beta, status)
