@@ -306,14 +306,16 @@ __global__ void __launch_bounds__(kRegThreads, 1) step_scores_reg_kernel(StepArg
                 cn += wcnt[w * a.max_steps + k];
             }
         u[k] = cn > 0 ? (double)t / (scale * (double)cn) : 0.0;
+        reinterpret_cast<float *>(cnt)[k] = (float)u[k];  // the blend's fp32 utility, over the count just read
     }
     __syncthreads();
+    const float *uf = reinterpret_cast<const float *>(cnt);
     float *o = a.out + (int64_t)row * c.max_slots;
     const float w = 1.f - a.beta;
 #pragma unroll
     for (int j = 0; j < kRegSlots; ++j) {
         const int i = tid + j * kRegThreads;
-        if (i < n) o[i] = fmaf(a.beta, (float)u[sid[i]], w * v[j]);
+        if (i < n) o[i] = fmaf(a.beta, uf[sid[i]], w * v[j]);
     }
 }
 
