@@ -56,7 +56,10 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int B = a.num_beacons, D = a.head_dim, Hq = a.num_q_heads;
     const int R = min(64, kPairs / B);                                   // queries per round of distances
-    const int DP = D + 1;                                                // padded row: rows fall in different banks
+    // padded rows: rows fall in different banks; with D % 4 == 0 the rows stay 16-byte aligned (4 floats of
+    // padding) so that the distance sums read four dimensions per load
+    const bool vec = (D & 3) == 0;
+    const int DP = vec ? D + 4 : D + 1;
     float *cb = reinterpret_cast<float *>(smem_raw);                   // [B][DP] beacons
     float *qs = cb + B * DP;                                             // [stage_rows][DP] staged queries
     float *dist = qs + (size_t)a.stage_rows * DP;                        // [R][B] distances of a round
@@ -76,9 +79,14 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
     auto qidx = [&](int j, int d) -> int64_t { return (((int64_t)sl * a.max_q + j) * Hq + h) * D + d; };
     auto qval = [&](int j, int d) -> float { return staged ? qs[(size_t)j * DP + d] : load_q(a, qidx(j, d)); };
 
-    for (int i = tid; i < B * D; i += kThreads) cb[(i / D) * DP + i % D] = gb[i];
+    // row-by-row copies (a warp per row, the lanes over the dimensions): no index division per element
+    for (int b = warp; b < B; b += kThreads / 32)
+        for (int d = lane; d < D; d += 32) cb[b * DP + d] = gb[b * D + d];
     if (staged)
-        for (int i = tid; i < m * D; i += kThreads) qs[(size_t)(i / D) * DP + i % D] = load_q(a, qidx(i / D, i % D));
+        for (int j = warp; j < m; j += kThreads / 32) {
+            const int64_t q0 = qidx(j, 0);
+            for (int d = lane; d < D; d += 32) qs[(size_t)j * DP + d] = load_q(a, q0 + d);
+        }
     if (tid < B) {
         cnt[tid] = gc[tid];
         drawn[tid] = 0;
@@ -100,10 +108,9 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
         }
     }
     __syncthreads();
-    for (int i = tid; i < B * D; i += kThreads) {
-        const int b = i / D, d = i % D;
-        if (seeded_from[b] >= 0) cb[b * DP + d] = qval(seeded_from[b], d);
-    }
+    for (int b = warp; b < B; b += kThreads / 32)
+        if (seeded_from[b] >= 0)
+            for (int d = lane; d < D; d += 32) cb[b * DP + d] = qval(seeded_from[b], d);
     __syncthreads();
 
     // 2. assignment, R queries per round; each thread runs up to four distance sums side by side, every one
@@ -112,7 +119,10 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
         const int nj = min(R, m - j0);
         const float *qb = qs + (size_t)j0 * DP;
         if (!staged) {
-            for (int i = tid; i < nj * D; i += kThreads) qs[(i / D) * DP + i % D] = load_q(a, qidx(j0 + i / D, i % D));
+            for (int jl = warp; jl < nj; jl += kThreads / 32) {
+                const int64_t q0 = qidx(j0 + jl, 0);
+                for (int d = lane; d < D; d += 32) qs[(size_t)jl * DP + d] = load_q(a, q0 + d);
+            }
             qb = qs;
             __syncthreads();
         }
@@ -125,11 +135,29 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
             qo[u] = (p / B) * DP;
             co[u] = (p % B) * DP;
         }
-        for (int d = 0; d < D; ++d) {
+        if (vec) {
+            for (int d = 0; d < D; d += 4) {  // the same order of operations, four dimensions per load
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float t = __fsub_rn(qb[qo[u] + d], cb[co[u] + d]);
-                acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                for (int u = 0; u < 4; ++u) {
+                    const float4 x = *reinterpret_cast<const float4 *>(qb + qo[u] + d);
+                    const float4 y = *reinterpret_cast<const float4 *>(cb + co[u] + d);
+                    float t = __fsub_rn(x.x, y.x);
+                    acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                    t = __fsub_rn(x.y, y.y);
+                    acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                    t = __fsub_rn(x.z, y.z);
+                    acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                    t = __fsub_rn(x.w, y.w);
+                    acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                }
+            }
+        } else {
+            for (int d = 0; d < D; ++d) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float t = __fsub_rn(qb[qo[u] + d], cb[co[u] + d]);
+                    acc[u] = __fadd_rn(acc[u], __fmul_rn(t, t));
+                }
             }
         }
 #pragma unroll
@@ -178,31 +206,34 @@ __global__ void __launch_bounds__(kThreads) beacon_kernel(BeaconArgs a) {
         }
         __syncthreads();
     }
-    for (int i = tid; i < B * D; i += kThreads) {
-        const int b = i / D, d = i % D;
+    for (int b = warp; b < B; b += kThreads / 32) {
         if (drawn[b] == 0) continue;  // a beacon that drew nothing keeps its value exactly
-        float s = __fmul_rn(cb[b * DP + d], (float)cnt[b]);
-        if (lists) {
-            for (int t = 0; t < drawn[b]; ++t) s = __fadd_rn(s, qval(list[first[b] + t], d));
-        } else {
-            for (int j = 0; j < m; ++j)
-                if (asg[j] == b) s = __fadd_rn(s, load_q(a, qidx(j, d)));
+        for (int d = lane; d < D; d += 32) {
+            float s = __fmul_rn(cb[b * DP + d], (float)cnt[b]);
+            if (lists) {
+                for (int t = 0; t < drawn[b]; ++t) s = __fadd_rn(s, qval(list[first[b] + t], d));
+            } else {
+                for (int j = 0; j < m; ++j)
+                    if (asg[j] == b) s = __fadd_rn(s, load_q(a, qidx(j, d)));
+            }
+            cb[b * DP + d] = __fdiv_rn(s, (float)(cnt[b] + drawn[b]));
         }
-        cb[b * DP + d] = __fdiv_rn(s, (float)(cnt[b] + drawn[b]));
     }
     __syncthreads();
-    for (int i = tid; i < B * D; i += kThreads) gb[i] = cb[(i / D) * DP + i % D];
+    for (int b = warp; b < B; b += kThreads / 32)
+        for (int d = lane; d < D; d += 32) gb[b * D + d] = cb[b * DP + d];
     if (tid < B) gc[tid] = cnt[tid] + drawn[tid];
     if (a.beacon_q) {
         // the beacons as the first rows of a query set [seq][layer][out_max_q][Hq][D]
-        for (int i = tid; i < B * D; i += kThreads) {
-            const int b = i / D, d = i % D;
-            const int64_t o = (((int64_t)sl * a.out_max_q + b) * Hq + h) * D + d;
-            const float v = cb[b * DP + d];
-            if (a.bf16)
-                static_cast<__nv_bfloat16 *>(a.beacon_q)[o] = __float2bfloat16_rn(v);
-            else
-                static_cast<float *>(a.beacon_q)[o] = v;
+        for (int b = warp; b < B; b += kThreads / 32) {
+            const int64_t o0 = (((int64_t)sl * a.out_max_q + b) * Hq + h) * D;
+            for (int d = lane; d < D; d += 32) {
+                const float v = cb[b * DP + d];
+                if (a.bf16)
+                    static_cast<__nv_bfloat16 *>(a.beacon_q)[o0 + d] = __float2bfloat16_rn(v);
+                else
+                    static_cast<float *>(a.beacon_q)[o0 + d] = v;
+            }
         }
     }
 }
@@ -215,13 +246,14 @@ cudaError_t launch_beacon(const void *q, const int32_t *num_q, int32_t num_seqs,
                           cudaStream_t stream) {
     // fixed part: beacons, a round of distances, the lists, the assignments; the rest stages queries (at
     // least one round of them, all of a group's when they fit)
-    const size_t fixed = (size_t)num_beacons * (head_dim + 1) * 4 + (size_t)kPairs * 4 + (size_t)kListMax * 2 +
+    const int dp = head_dim % 4 == 0 ? head_dim + 4 : head_dim + 1;  // the kernel's padded row (DP)
+    const size_t fixed = (size_t)num_beacons * dp * 4 + (size_t)kPairs * 4 + (size_t)kListMax * 2 +
                          (((size_t)max_q + 15) & ~(size_t)15);
     const int round_rows = std::min(64, kPairs / num_beacons);
     const size_t room = kSmemCap - 2048 - fixed;  // static shared memory and slack
-    int rows = (int)std::min<size_t>((size_t)max_q, room / ((size_t)(head_dim + 1) * 4));
+    int rows = (int)std::min<size_t>((size_t)max_q, room / ((size_t)dp * 4));
     rows = std::max(rows, round_rows);
-    const size_t smem = fixed + (size_t)rows * (head_dim + 1) * 4;
+    const size_t smem = fixed + (size_t)rows * dp * 4;
     if (smem > kSmemCap - 2048) return cudaErrorInvalidValue;
     static int smem_set[kMaxDevices];
     cudaError_t e = dyn_smem_at_least((const void *)beacon_kernel, smem, smem_set);

@@ -42,9 +42,10 @@ def _run(q, num_q, beacons, counts, beacon_q=None):
     assert st.tolist() == [0, 0]
 
 
-@pytest.mark.parametrize("dtype,D,B", [(torch.bfloat16, 128, 16), (torch.float32, 64, 64)])
+@pytest.mark.parametrize("dtype,D,B", [(torch.bfloat16, 128, 16), (torch.float32, 64, 64), (torch.float32, 37, 8)])
 def test_rounds_match_oracle_bitwise(dtype, D, B):
-    """Several rounds with state carried: uneven query counts (one below B, one zero), beacons exact."""
+    """Several rounds with state carried: uneven query counts (one below B, one zero), beacons exact.  A head size
+    that is not a multiple of 4 takes the distance sums one dimension per load."""
     gen = torch.Generator().manual_seed(7)
     S, L, Hq, max_q = 3, 2, 4, 96
     beacons = torch.zeros((S, L, Hq, B, D), device=DEV)
