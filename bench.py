@@ -521,15 +521,18 @@ def cpu_baseline(config, rows, ratchet_steps, budget):
             "seconds": t_par, "host_cores": cores}
 
 
-def config_spec(config):
-    """The workload of a bench configuration (seeded; the same spec on the GPU side and in the oracle's sample)."""
+def config_spec(config, seqs=None, layers=None):
+    """The workload of a bench configuration (seeded; the same spec on the GPU side and in the oracle's sample).
+    seqs / layers shrink batch16 and stress to fewer sequences or layers of the same rows (a case small enough
+    for an ncu capture)."""
     from agent_kv_cache_lse_b200 import synth
+    size = {k: v for k, v in (("num_seqs", seqs), ("num_layers", layers)) if v is not None}
     if config == "llama8b":
         return synth.llama8b_layer()
     if config == "batch16":
-        return synth.batch16()
+        return synth.batch16(**size)
     if config == "stress":
-        return synth.stress()
+        return synth.stress(**size)
     if config == "streaming":
         return synth.streaming()
     raise ValueError(config)
@@ -597,7 +600,7 @@ def run_config(args, device):
     from agent_kv_cache_lse_b200.round import EvictionRound
     hbm, tf_burst, tf_sus, peak_kind = peaks()
     name = args.config
-    spec = config_spec(name)
+    spec = config_spec(name, args.seqs, args.layers)
     layout = synth.make_layout(spec)
     stress = name == "stress"
     if stress:
@@ -680,14 +683,17 @@ def run_config(args, device):
     sample = sorted(int(x) for x in rng.choice(spec.rows, size=8, replace=False))
     steps_share = 0 if stress else max(1, round(spec.logits_steps * spec.num_seqs / spec.rows))
     del pristine
-    cpu = None if args.no_cpu else cpu_baseline(name, sample, steps_share, budget)
+    reduced = args.seqs is not None or args.layers is not None  # a smaller case: no oracle leg
+    cpu = None if args.no_cpu or reduced else cpu_baseline(name, sample, steps_share, budget)
     return {
         "metric": f"KV entries scored+compacted/sec ({name} workload)", "value": work["entries"] / (ms_step / 1e3),
         "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "ms_per_step_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; " + ("torch N(0,1) pools" if stress else "counter-based generator") + ")",
-        "config": {"workload": CONFIG_TEXT[name], "entries_per_step": work["entries"], "rows": spec.rows,
+        "config": {"workload": CONFIG_TEXT[name] if args.seqs is None and args.layers is None else
+                   f"{CONFIG_TEXT[name]}, reduced to {spec.num_seqs} sequences x {spec.num_layers} layers",
+                   "entries_per_step": work["entries"], "rows": spec.rows,
                    "queries": int(queries.num_q.sum()), "budget": "ratchet" if logits is not None else budget,
                    "l2": "flushed (256 MB write) before every step; inputs far larger than L2"},
         "roofline": {"kernel": "score_tc_kernel (kvc_score_from_lse)", "bound": "tensor", "achieved": achieved,
@@ -1180,6 +1186,8 @@ def main():
     ap.add_argument("--config", default="llama8b", choices=["llama8b", "batch16", "stress", "streaming"],
                     help="workload of the round (llama8b is the headline line)")
     ap.add_argument("--rounds", type=int, default=200, help="rounds of the streaming workload")
+    ap.add_argument("--seqs", type=int, default=None, help="batch16 / stress: fewer sequences (a smaller case)")
+    ap.add_argument("--layers", type=int, default=None, help="batch16 / stress: fewer layers (a smaller case)")
     ap.add_argument("--kvstreams", action="store_true", help="the streaming workload carried across rollouts")
     ap.add_argument("--rollouts", type=int, default=5, help="rollouts of the --kvstreams line")
     args = ap.parse_args()
