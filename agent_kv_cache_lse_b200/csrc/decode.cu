@@ -68,6 +68,7 @@ constexpr int kMaxGroup = 8;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxD = 128;
 constexpr int kMaxRing = 4;                 // stages per warp
+constexpr int kOrderRows = 1024;            // rows up to this many are taken longest first
 constexpr int kTmRing = 3;                  // stages per warp with the logits in TMEM
 constexpr int kTmMinCluster = 1;            // smallest cluster of the TMEM plan
 constexpr float kLn2 = 0.6931471805599453f;
@@ -86,6 +87,7 @@ struct DecodeArgs {
     int32_t slice_cap;    // slots per CTA the logits buffer holds (multiple of CH)
     float scale_log2;     // log2(e) / sqrt(D)
     int32_t *status;
+    int32_t order_rows;   // clusters take the rows longest first (rows <= kOrderRows)
 };
 
 struct DecodeShared {
@@ -213,10 +215,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     __shared__ DecodeShared sh;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank(), C = (int)cl.num_blocks();
-    const int row = blockIdx.x / C;
     const CacheView &c = a.c;
-    const int G = a.group, Hkv = c.num_kv_heads, CH = a.chunk, P = c.page_size;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the cluster's row: the one at its index, or (order_rows) the one whose length ranks there, longest first
+    // (ties by row index), so that the longest rows start first and the launch ends evenly; every CTA of the
+    // cluster ranks the same lengths and picks the same row
+    int row_pick = blockIdx.x / C;
+    if (a.order_rows) {
+        int *lens = reinterpret_cast<int *>(smem);  // the stages are not in use yet
+        __shared__ int picked;
+        const int R = c.rows;
+        for (int r = tid; r < R; r += kThreads) {
+            const int n = c.row_len[r];
+            lens[r] = (n < 0 || n > c.max_slots) ? 0 : n;
+        }
+        __syncthreads();
+        for (int r = tid; r < R; r += kThreads) {
+            const int n = lens[r];
+            int above = 0;
+            for (int q = 0; q < R; ++q) {
+                const int m = lens[q];
+                above += (m > n || (m == n && q < r)) ? 1 : 0;
+            }
+            if (above == row_pick) picked = r;
+        }
+        __syncthreads();
+        row_pick = picked;
+    }
+    const int row = row_pick;
+    const int G = a.group, Hkv = c.num_kv_heads, CH = a.chunk, P = c.page_size;
     const int seq = row / (c.num_layers * Hkv), layer = (row / Hkv) % c.num_layers, kvh = row % Hkv;
     const uint32_t half = (uint32_t)CH * D * sizeof(T);   // bytes of a chunk's K (or V)
     // a stage: the chunk's K and V rows, then (TMEM logits) its CH slot positions and CH old scores
@@ -921,8 +948,10 @@ cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, in
     static int smem_set[kMaxDevices];
     cudaError_t e = dyn_smem_at_least((const void *)decode_kernel<T, D, GM, RW, TM, MM>, p.smem, smem_set);
     if (e != cudaSuccess) return e;
+    const int sms = device_sms();
+    const int order = c.rows <= kOrderRows && (int64_t)c.rows * p.C > sms ? 1 : 0;  // more than one wave
     DecodeArgs a{c, q, q_pos, num_q_heads, G, out, lse, scores, accumulate ? 1 : 0, p.CH, p.RW, p.cap,
-                 (float)(1.4426950408889634 / std::sqrt((double)D)), status};
+                 (float)(1.4426950408889634 / std::sqrt((double)D)), status, order};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(c.rows * p.C));
     cfg.blockDim = dim3(kThreads);
