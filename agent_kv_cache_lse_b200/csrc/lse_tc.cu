@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace cg = cooperative_groups;
 
@@ -450,34 +451,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_lse() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 template <int D>
 cudaError_t launch_lse_tc_t(const CacheView &c, const QueryView &q, int32_t *status, cudaStream_t stream) {
     using PL = LPlan<D>;
-    auto enc = encode_fn_lse();
-    if (!enc) return cudaErrorNotSupported;
+    if (!tmap_encoder()) return cudaErrorNotSupported;
     const int G = q.group, nqt = kCols / G;
     CUtensorMap tk, tq;
     {
         cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.num_pages * 16};
         cuuint64_t strides[1] = {(cuuint64_t)D * 2};
         cuuint32_t box[2] = {64, 16};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(c.k_pool), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+        if (tmap_bf16(kTmapLseK, &tk, 2, c.k_pool, dims, strides, box) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)q.num_q_heads, (cuuint64_t)q.max_q,
@@ -485,11 +469,7 @@ cudaError_t launch_lse_tc_t(const CacheView &c, const QueryView &q, int32_t *sta
         cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)q.num_q_heads * D * 2,
                                  (cuuint64_t)q.max_q * q.num_q_heads * D * 2};
         cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)nqt, 1};
-        cuuint32_t es[4] = {1, 1, 1, 1};
-        if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q.q), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+        if (tmap_bf16(kTmapLseQ, &tq, 4, q.q, dims, strides, box) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
     LseTcArgs args;
     args.c = c;

@@ -46,6 +46,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tmap.h"
 
 namespace kvc {
 namespace {
@@ -1025,24 +1026,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
 
 template <int D>
 cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool accumulate, int32_t *status,
                      cudaStream_t stream, char *err, size_t errlen) {
     using PL = Plan<D>;
-    auto enc = encode_fn();
-    if (!enc) {
+    if (!tmap_encoder()) {
         snprintf(err, errlen, "cuTensorMapEncodeTiled unavailable");
         return cudaErrorNotSupported;
     }
@@ -1057,10 +1046,7 @@ cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool
         cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.num_pages * 16};
         cuuint64_t strides[1] = {(cuuint64_t)D * 2};
         cuuint32_t box[2] = {64, 16};
-        cuuint32_t es[2] = {1, 1};
-        CUresult r = enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(c.k_pool), dims, strides, box, es,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        CUresult r = tmap_bf16(kTmapScoreK, &tk, 2, c.k_pool, dims, strides, box);
         if (r != CUDA_SUCCESS) {
             snprintf(err, errlen, "K tensor map encode failed (%d)", (int)r);
             return cudaErrorInvalidValue;
@@ -1073,10 +1059,7 @@ cudaError_t launch_t(const CacheView &c, const QueryView &q, float *scores, bool
         cuuint64_t strides[3] = {(cuuint64_t)q.num_q_heads * D * 2, (cuuint64_t)D * 2,
                                  (cuuint64_t)q.max_q * q.num_q_heads * D * 2};
         cuuint32_t box[4] = {64, (cuuint32_t)nqb, (cuuint32_t)G, 1};
-        cuuint32_t es[4] = {1, 1, 1, 1};
-        CUresult r = enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q.q), dims, strides, box, es,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        CUresult r = tmap_bf16(kTmapScoreQ, &tq, 4, q.q, dims, strides, box);
         if (r != CUDA_SUCCESS) {
             snprintf(err, errlen, "Q tensor map encode failed (%d)", (int)r);
             return cudaErrorInvalidValue;
