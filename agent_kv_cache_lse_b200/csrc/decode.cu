@@ -34,7 +34,7 @@
 // its old scores (stored to TMEM beside the logits).  Shared memory then holds only the K/V stages, so
 // every warp keeps two chunks in flight instead of one, and the final scores need no global reads.
 //
-// With bf16 K/V, four-head groups (G' = 4) and 16-slot chunks, a chunk's two contractions run on the
+// With bf16 K/V, groups of four or eight heads (G' = 4, 8) and 16-slot chunks, a chunk's two contractions run on the
 // tensor cores as warp-level mma tiles (m16n8k16, fp32 accumulate) instead of per-lane FMAs:
 //   * S = K Q^T: the 16 keys are the tile's rows, D its k-steps, the group's heads (padded to 8) its
 //     columns; K comes from the stage with ldmatrix (each key row's 16-byte pieces XOR-swizzled by the
@@ -47,7 +47,8 @@
 //     products keep 16 bits of P's mantissa, and reaches the B-operand layout by an 8x8 register
 //     transpose (movmatrix) of the S accumulator's [key][head] pairs.
 // A lane then holds the heads 2 (lane % 4), + 1 of keys lane / 4 and lane / 4 + 8; the kept logits go to
-// TMEM two to a lane (the lanes with bit 1 set take the second key from lane ^ 2).
+// TMEM two to a lane at G' = 4 (the lanes with bit 1 set take the second key from lane ^ 2, the other lanes'
+// heads being padding) and all four at G' = 8.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -201,13 +202,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     constexpr int MAXSTEPS = 16 / KW;
     // reduce-scatter of the dot products when every lane can end with whole ones and the partials fit
     constexpr bool kRS = MAXSTEPS * GM >= LK && MAXSTEPS * GM <= 32;
-    static_assert(!TM || (kRS && LK == 2 * MAXSTEPS), "TMEM logits need the reduce-scatter with two lanes per key");
-    // TMEM logits: a lane keeps RL logits per chunk (two lanes per key), in columns [i * RL, i * RL + RL) of
-    // its warp's 256; the old scores sit in columns kTmCap * RL + i
-    constexpr int RL = kRS ? MAXSTEPS * GM / LK : 1;
+    static_assert(!TM || MM || (kRS && LK == 2 * MAXSTEPS),
+                  "TMEM logits need the reduce-scatter with two lanes per key, or the tensor-core chunks");
+    // MM: the chunk's two contractions on the tensor cores (bf16, groups of 4 or 8 heads, 16-slot chunks, logits
+    // in TMEM)
+    static_assert(!MM || (TM && (GM == 4 || GM == 8) && sizeof(T) == 2), "tensor-core chunks: bf16, G' = 4 or 8");
+    // TMEM logits: a lane keeps RL logits per chunk in columns [i * RL, i * RL + RL) of its warp's 256, and the
+    // old score it adds in column kTmCap * RL + i: two lanes per key (reduce-scatter, or MM at G' = 4, RL =
+    // G' / 2), or (MM at G' = 8) four lanes per pair of keys, RL = 4
+    constexpr int RL = MM ? GM / 2 : (kRS ? MAXSTEPS * GM / LK : 1);
     constexpr int kTmCap = (256 / (RL + 1)) / 8 * 8;  // chunks per warp the columns hold (a multiple of 8)
-    // MM: the chunk's two contractions on the tensor cores (bf16, four-head groups, 16-slot chunks, logits in TMEM)
-    static_assert(!MM || (TM && GM == 4 && sizeof(T) == 2 && RL == 2), "tensor-core chunks: bf16, G' = 4, TMEM");
     constexpr int RB = D * (int)sizeof(T);  // bytes of a key's row
     constexpr int NS = D / 16;              // k-steps of q . k, 16-row tiles of the output
     constexpr float kSlack = 8.f;           // MM: the running maximum moves only when a logit passes it by 8 (log2)
@@ -448,14 +452,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             ms[0] += p00 + p10;
             ms[1] += p01 + p11;
             if constexpr (TM) {
-                if (a.scores) {  // logits of key ka (+ 8 on lanes with bit 1 set, taken from lane ^ 2), old score
-                    const bool up = (lane & 2) != 0;
-                    const float x0 = __shfl_xor_sync(0xffffffffu, l10, 2), x1 = __shfl_xor_sync(0xffffffffu, l11, 2);
-                    const float lv[2] = {up ? x0 : l00, up ? x1 : l01};
-                    tm_st(tmw + (uint32_t)(i * 2), lv);
-                    if (acc_old) {
-                        const float ov[1] = {reinterpret_cast<const float *>(psS + CH)[ka + (up ? 8 : 0)]};
-                        tm_st(tmw + (uint32_t)(kTmCap * 2 + i), ov);
+                if (a.scores) {
+                    if constexpr (GM == 4) {  // key ka (+ 8 on lanes with bit 1 set, taken from lane ^ 2), old score
+                        const bool up = (lane & 2) != 0;
+                        const float x0 = __shfl_xor_sync(0xffffffffu, l10, 2), x1 = __shfl_xor_sync(0xffffffffu, l11, 2);
+                        const float lv[2] = {up ? x0 : l00, up ? x1 : l01};
+                        tm_st(tmw + (uint32_t)(i * RL), lv);
+                        if (acc_old) {
+                            const float ov[1] = {reinterpret_cast<const float *>(psS + CH)[ka + (up ? 8 : 0)]};
+                            tm_st(tmw + (uint32_t)(kTmCap * RL + i), ov);
+                        }
+                    } else {  // all eight heads are real: keys ka and ka + 8, heads hm, hm + 1; old score of ka (+ 8)
+                        const float lv[4] = {l00, l01, l10, l11};
+                        tm_st(tmw + (uint32_t)(i * RL), lv);
+                        if (acc_old) {
+                            const float ov[1] = {reinterpret_cast<const float *>(psS + CH)[ka + ((lane & 1) ? 8 : 0)]};
+                            tm_st(tmw + (uint32_t)(kTmCap * RL + i), ov);
+                        }
                     }
                 }
             }
@@ -774,7 +787,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             if (bad) report(a.status, KVC_DEV_BAD_PAGE, row);
         }
     }
-    if (MM && a.scores) {
+    if (MM && GM == 8 && a.scores) {
+        // lane L holds keys L / 4 and L / 4 + 8, heads 2 (L % 4), + 1: the four lanes of L / 4 sum both keys'
+        // heads; lane 4 (L / 4) writes the first key, lane 4 (L / 4) + 1 the second (the one whose old score it kept)
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        const int hm = 2 * (lane & 3);
+        float inv[2], mg[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            inv[r] = (hm + r < G && sh.S[hm + r] > 0.f) ? 1.f / sh.S[hm + r] : 0.f;
+            mg[r] = sh.M[hm + r];
+        }
+        const int ko = (lane >> 2) + ((lane & 1) ? 8 : 0);
+        float *sc = a.scores + (int64_t)row * c.max_slots + lo;
+        for (int i0 = 0; i0 < ni; i0 += 8) {
+            uint32_t lr[32], orr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int b = 0; b < 4; ++b) tm_ld8(tmw + (uint32_t)(i0 * RL + 8 * b), lr + 8 * b);
+            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * RL + i0), orr);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int b = 0; b < 4; ++b) tm_hold8(lr + 8 * b);
+            tm_hold8(orr);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float pa = 0.f, pb = 0.f;
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                    if (hm + r < G) {
+                        pa = fmaf(weight(__uint_as_float(lr[4 * b + r]), mg[r]), inv[r], pa);
+                        pb = fmaf(weight(__uint_as_float(lr[4 * b + 2 + r]), mg[r]), inv[r], pb);
+                    }
+                pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+                pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 2);
+                const int il = (warp + (i0 + b) * kWarps) * CH + ko;
+                if (i0 + b < ni && (lane & 3) < 2 && il < cnt)
+                    sc[il] = __uint_as_float(orr[b]) + ((lane & 1) ? pb : pa);
+            }
+        }
+    }
+    if (MM && GM == 4 && a.scores) {
         // lane L holds key (L / 4) + 8 ((L >> 1) & 1), heads 2 (L & 1), + 1: the pair L, L ^ 1 sums the key's heads
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         const int hl = 2 * (lane & 1);
@@ -788,9 +842,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         float *sc = a.scores + (int64_t)row * c.max_slots + lo;
         for (int i0 = 0; i0 < ni; i0 += 8) {
             uint32_t lr[16], orr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            tm_ld8(tmw + (uint32_t)(i0 * 2), lr);
-            tm_ld8(tmw + (uint32_t)(i0 * 2 + 8), lr + 8);
-            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * 2 + i0), orr);
+            tm_ld8(tmw + (uint32_t)(i0 * RL), lr);
+            tm_ld8(tmw + (uint32_t)(i0 * RL + 8), lr + 8);
+            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * RL + i0), orr);
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             tm_hold8(lr);
             tm_hold8(lr + 8);
@@ -900,24 +954,29 @@ constexpr bool two_lanes_per_key(int D, int GM) {
 //
 // With `aligned` (slot positions and scores 16-byte aligned) and the two-lanes-per-key reduce-scatter, the
 // TMEM plan comes first: three stages per warp, the smallest cluster whose warps' chunks fit the TMEM columns.
-// With bf16, G' = 4, 16-slot chunks and a 4-byte aligned query (`q4`), the chunks' contractions run as mma tiles.
+// With bf16, G' = 4 or 8, 16-slot chunks and a 4-byte aligned query (`q4`), the chunks' contractions run as mma
+// tiles (their TMEM layout needs no reduce-scatter).
 Plan plan_for(const CacheView &c, int G, int sms, bool aligned, bool q4) {
     const size_t elem = c.dtype == KVC_BF16 ? 2 : 4;
     const size_t partial = (size_t)kWarps * G * c.head_dim * 4;
     const int GM = group_bound(G);
     int C0 = 1;
     while (C0 < kMaxCluster && (int64_t)c.rows * C0 < sms) C0 <<= 1;
-    if (aligned && two_lanes_per_key(c.head_dim, GM)) {
-        const int RL = GM / 2, cap_w = (256 / (RL + 1)) / 8 * 8;
+    const bool two = two_lanes_per_key(c.head_dim, GM);
+    const bool mm_ok = q4 && c.dtype == KVC_BF16 && (GM == 4 || GM == 8);  // tensor-core chunks (16-slot ones)
+    if (aligned && (two || mm_ok)) {
+        const int RL = GM / 2, cap_w = (256 / (RL + 1)) / 8 * 8;  // the kernel's RL and kTmCap
         for (int CH = std::min(16, c.page_size); CH >= 4; --CH) {
             if (c.page_size % CH || CH % 4 || c.max_slots % CH) continue;
+            const bool mm = mm_ok && CH == 16;
+            if (!mm && !two) continue;
             const size_t stage = 2 * (size_t)CH * c.head_dim * elem + 8 * (size_t)CH;
             const size_t smem = (size_t)kTmRing * kWarps * stage;
             if (smem > kSmemLimitTm || smem < partial) continue;
             const int64_t nch = (c.max_slots + CH - 1) / CH;
             for (int C = std::max(C0, kTmMinCluster); C <= kMaxCluster; C <<= 1)
                 if (((nch + C - 1) / C + kWarps - 1) / kWarps <= cap_w)
-                    return Plan{C, CH, kTmRing, 0, smem, true, q4 && c.dtype == KVC_BF16 && GM == 4 && CH == 16};
+                    return Plan{C, CH, kTmRing, 0, smem, true, mm};
         }
     }
     for (int CH = std::min(16, c.page_size); CH >= 1; --CH) {
@@ -970,12 +1029,12 @@ cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, in
 template <typename T, int D, int GM>
 cudaError_t launch_r(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                      float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, const Plan &p) {
+    if constexpr ((GM == 4 || GM == 8) && sizeof(T) == 2) {
+        if (p.mm)
+            return launch_t<T, D, GM, kTmRing, true, true>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
+                                                           status, stream, p);
+    }
     if constexpr (two_lanes_per_key(D, GM)) {
-        if constexpr (GM == 4 && sizeof(T) == 2) {
-            if (p.mm)
-                return launch_t<T, D, GM, kTmRing, true, true>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
-                                                               status, stream, p);
-        }
         if (p.tm && !p.mm)
             return launch_t<T, D, GM, kTmRing, true, false>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
                                                             status, stream, p);

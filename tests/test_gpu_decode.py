@@ -96,6 +96,7 @@ CASES = {
     "gqa8_d64": dict(Hq=16, Hkv=2, D=64, ctx=(2500,), seed=35),
     "gqa4_d64": dict(Hq=8, Hkv=2, D=64, ctx=(2222, 999), S=2, seed=46),
     "gqa3": dict(Hq=24, Hkv=8, ctx=(1800,), seed=47),
+    "gqa8_d128": dict(Hq=64, Hkv=8, ctx=(3001, 1234), S=2, seed=49),
     "gqa2_f32": dict(Hq=4, Hkv=2, dtype="f32", ctx=(1111,), seed=36),
     "short_rows": dict(S=2, ctx=(17, 300), seed=37),
 }
