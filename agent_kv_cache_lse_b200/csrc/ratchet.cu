@@ -285,8 +285,10 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
     }
     cluster.sync();
     if (rank == 0) {
-        // merge the cluster: LSE from the (max, sum) pairs; the sum of the k largest from the sorted lists
-        __shared__ float allv[kCluster * kMaxTopK];
+        // merge the cluster: LSE from the (max, sum) pairs; the sum of the k largest from the sorted lists,
+        // gathered into the exact fallback's histogram (free again by now) when they fit, else read in place
+        float *allv = reinterpret_cast<float *>(sh.hist);
+        const bool gathered = K * kCluster <= 256;
         __shared__ float pm[kCluster];
         __shared__ double ps[kCluster];
         __shared__ int anybad;
@@ -296,7 +298,8 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
             ps[tid] = peer->csum;
             if (tid == 0) anybad = 0;
         }
-        for (int e = tid; e < kCluster * K; e += kThreads) allv[e] = cluster.map_shared_rank(&sh, e / K)->topk[e % K];
+        if (gathered)
+            for (int e = tid; e < kCluster * K; e += kThreads) allv[e] = cluster.map_shared_rank(&sh, e / K)->topk[e % K];
         __syncthreads();
         if (tid < kCluster && cluster.map_shared_rank(&sh, tid)->nbad) atomicOr(&anybad, 1);
         if (warp == 0) {
@@ -304,7 +307,9 @@ __global__ void __launch_bounds__(kThreads) confidence_kernel(ConfArgs a) {
             int head = 0;
             double topsum = 0.0;
             for (int t = 0; t < K; ++t) {
-                const float hv = (lane < kCluster && head < K) ? allv[lane * K + head] : -INFINITY;
+                const float hv = (lane < kCluster && head < K)
+                                     ? (gathered ? allv[lane * K + head] : cluster.map_shared_rank(&sh, lane)->topk[head])
+                                     : -INFINITY;
                 float best = hv;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
