@@ -21,9 +21,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def spec_of(S=1, L=1, Hq=32, Hkv=8, D=128, ctx=(4096 + 99,), dtype="bf16", seed=31, heavy=0.02):
+def spec_of(S=1, L=1, Hq=32, Hkv=8, D=128, ctx=(4096 + 99,), dtype="bf16", seed=31, heavy=0.02, P=16):
     return synth.Spec(name="decode", seed=seed, num_seqs=S, num_layers=L, num_q_heads=Hq, num_kv_heads=Hkv,
-                      head_dim=D, dtype=dtype, ctx=list(ctx), budget=512, heavy_frac=heavy)
+                      head_dim=D, dtype=dtype, ctx=list(ctx), budget=512, heavy_frac=heavy, page_size=P)
 
 
 def decode_inputs(w, q_pos=None):
@@ -97,6 +97,12 @@ CASES = {
     "gqa4_d64": dict(Hq=8, Hkv=2, D=64, ctx=(2222, 999), S=2, seed=46),
     "gqa3": dict(Hq=24, Hkv=8, ctx=(1800,), seed=47),
     "gqa8_d128": dict(Hq=64, Hkv=8, ctx=(3001, 1234), S=2, seed=49),
+    # 8-token pages: 8-slot chunks, so the dot products run on the FMA pipes with the logits in TMEM (G = 4)
+    # and in shared memory (G = 8)
+    "pages8_gqa4": dict(ctx=(2500, 777), S=2, seed=50, P=8),
+    "pages8_gqa8": dict(Hq=64, Hkv=8, ctx=(1900,), seed=51, P=8),
+    # 12-token pages: 12-slot chunks (not a power of two)
+    "pages12_gqa4": dict(ctx=(2000,), seed=52, P=12),
     "gqa2_f32": dict(Hq=4, Hkv=2, dtype="f32", ctx=(1111,), seed=36),
     "short_rows": dict(S=2, ctx=(17, 300), seed=37),
 }
