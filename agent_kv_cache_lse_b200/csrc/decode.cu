@@ -34,8 +34,8 @@
 // its old scores (stored to TMEM beside the logits).  Shared memory then holds only the K/V stages, so
 // every warp keeps two chunks in flight instead of one, and the final scores need no global reads.
 //
-// With bf16 K/V, groups of four or eight heads (G' = 4, 8) and 16-slot chunks, a chunk's two contractions run on the
-// tensor cores as warp-level mma tiles (m16n8k16, fp32 accumulate) instead of per-lane FMAs:
+// With bf16 K/V and 16-slot chunks, a chunk's two contractions run on the tensor cores as warp-level mma
+// tiles (m16n8k16, fp32 accumulate) instead of per-lane FMAs:
 //   * S = K Q^T: the 16 keys are the tile's rows, D its k-steps, the group's heads (padded to 8) its
 //     columns; K comes from the stage with ldmatrix (each key row's 16-byte pieces XOR-swizzled by the
 //     row index as the copies land, so an ldmatrix phase hits eight bank groups), Q sits in registers;
@@ -48,7 +48,8 @@
 //     transpose (movmatrix) of the S accumulator's [key][head] pairs.
 // A lane then holds the heads 2 (lane % 4), + 1 of keys lane / 4 and lane / 4 + 8; the kept logits go to
 // TMEM two to a lane at G' = 4 (the lanes with bit 1 set take the second key from lane ^ 2, the other lanes'
-// heads being padding) and all four at G' = 8.
+// heads being padding), all four at G' = 8, and one to each lane of a group at G' <= 2 (only the group's
+// first lane holds real heads).
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -206,11 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
                   "TMEM logits need the reduce-scatter with two lanes per key, or the tensor-core chunks");
     // MM: the chunk's two contractions on the tensor cores (bf16, groups of 4 or 8 heads, 16-slot chunks, logits
     // in TMEM)
-    static_assert(!MM || (TM && (GM == 4 || GM == 8) && sizeof(T) == 2), "tensor-core chunks: bf16, G' = 4 or 8");
+    static_assert(!MM || (TM && sizeof(T) == 2), "tensor-core chunks: bf16, logits in TMEM");
     // TMEM logits: a lane keeps RL logits per chunk in columns [i * RL, i * RL + RL) of its warp's 256, and the
-    // old score it adds in column kTmCap * RL + i: two lanes per key (reduce-scatter, or MM at G' = 4, RL =
-    // G' / 2), or (MM at G' = 8) four lanes per pair of keys, RL = 4
-    constexpr int RL = MM ? GM / 2 : (kRS ? MAXSTEPS * GM / LK : 1);
+    // old score it adds in column kTmCap * RL + i: two lanes per key (reduce-scatter, RL = G' / 2; MM at G' <= 2,
+    // RL = 1; MM at G' = 4, RL = 2), or (MM at G' = 8) four lanes per pair of keys, RL = 4
+    constexpr int RL = MM ? (GM <= 2 ? 1 : GM / 2) : (kRS ? MAXSTEPS * GM / LK : 1);
     constexpr int kTmCap = (256 / (RL + 1)) / 8 * 8;  // chunks per warp the columns hold (a multiple of 8)
     constexpr int RB = D * (int)sizeof(T);  // bytes of a key's row
     constexpr int NS = D / 16;              // k-steps of q . k, 16-row tiles of the output
@@ -453,7 +454,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             ms[1] += p01 + p11;
             if constexpr (TM) {
                 if (a.scores) {
-                    if constexpr (GM == 4) {  // key ka (+ 8 on lanes with bit 1 set, taken from lane ^ 2), old score
+                    if constexpr (GM <= 2) {
+                        // only lane 4 (lane / 4) holds real heads (0, 1): its four logits go one to each lane of
+                        // its group, lane L taking value L % 4 (key ka + 8 (L % 4 / 2), head L % 2)
+                        const int src = lane & ~3, v = lane & 3;
+                        const float x0 = __shfl_sync(0xffffffffu, l00, src), x1 = __shfl_sync(0xffffffffu, l01, src);
+                        const float x2 = __shfl_sync(0xffffffffu, l10, src), x3 = __shfl_sync(0xffffffffu, l11, src);
+                        const float lv[1] = {v == 0 ? x0 : v == 1 ? x1 : v == 2 ? x2 : x3};
+                        tm_st(tmw + (uint32_t)(i * RL), lv);
+                        if (acc_old) {
+                            const float ov[1] = {reinterpret_cast<const float *>(psS + CH)[ka + ((v & 2) ? 8 : 0)]};
+                            tm_st(tmw + (uint32_t)(kTmCap * RL + i), ov);
+                        }
+                    } else if constexpr (GM == 4) {  // key ka (+ 8 on lanes with bit 1 set, from lane ^ 2), old score
                         const bool up = (lane & 2) != 0;
                         const float x0 = __shfl_xor_sync(0xffffffffu, l10, 2), x1 = __shfl_xor_sync(0xffffffffu, l11, 2);
                         const float lv[2] = {up ? x0 : l00, up ? x1 : l01};
@@ -679,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             ms[0] += __shfl_xor_sync(0xffffffffu, ms[0], off);
             ms[1] += __shfl_xor_sync(0xffffffffu, ms[1], off);
         }
-        if (lane < GM / 2) {
+        if (lane < (GM + 1) / 2) {
             sh.wm[warp][2 * lane] = mm[0];
             sh.wm[warp][2 * lane + 1] = mm[1];
             sh.ws[warp][2 * lane] = ms[0];
@@ -785,6 +798,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             bool bad = false;
             for (int r = 0; r < C; ++r) bad |= cl.map_shared_rank(&sh, r)->bad != 0;
             if (bad) report(a.status, KVC_DEV_BAD_PAGE, row);
+        }
+    }
+    if (MM && GM <= 2 && a.scores) {
+        // lane L holds key L / 4 + 8 (L % 4 / 2), head L % 2: the pair L, L ^ 1 sums the key's heads
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        const int hh = lane & 1;
+        const float inv = (hh < G && sh.S[hh] > 0.f) ? 1.f / sh.S[hh] : 0.f, mg = sh.M[hh];
+        const int ko = (lane >> 2) + ((lane & 2) ? 8 : 0);
+        float *sc = a.scores + (int64_t)row * c.max_slots + lo;
+        for (int i0 = 0; i0 < ni; i0 += 8) {
+            uint32_t lr[8], orr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            tm_ld8(tmw + (uint32_t)(i0 * RL), lr);
+            if (acc_old) tm_ld8(tmw + (uint32_t)(kTmCap * RL + i0), orr);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            tm_hold8(lr);
+            tm_hold8(orr);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float part = hh < G ? weight(__uint_as_float(lr[b]), mg) * inv : 0.f;
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                const int il = (warp + (i0 + b) * kWarps) * CH + ko;
+                if (i0 + b < ni && hh == 0 && il < cnt) sc[il] = __uint_as_float(orr[b]) + part;
+            }
         }
     }
     if (MM && GM == 8 && a.scores) {
@@ -954,8 +990,8 @@ constexpr bool two_lanes_per_key(int D, int GM) {
 //
 // With `aligned` (slot positions and scores 16-byte aligned) and the two-lanes-per-key reduce-scatter, the
 // TMEM plan comes first: three stages per warp, the smallest cluster whose warps' chunks fit the TMEM columns.
-// With bf16, G' = 4 or 8, 16-slot chunks and a 4-byte aligned query (`q4`), the chunks' contractions run as mma
-// tiles (their TMEM layout needs no reduce-scatter).
+// With bf16, 16-slot chunks and a 4-byte aligned query (`q4`), the chunks' contractions run as mma tiles (their
+// TMEM layout needs no reduce-scatter).
 Plan plan_for(const CacheView &c, int G, int sms, bool aligned, bool q4) {
     const size_t elem = c.dtype == KVC_BF16 ? 2 : 4;
     const size_t partial = (size_t)kWarps * G * c.head_dim * 4;
@@ -963,9 +999,9 @@ Plan plan_for(const CacheView &c, int G, int sms, bool aligned, bool q4) {
     int C0 = 1;
     while (C0 < kMaxCluster && (int64_t)c.rows * C0 < sms) C0 <<= 1;
     const bool two = two_lanes_per_key(c.head_dim, GM);
-    const bool mm_ok = q4 && c.dtype == KVC_BF16 && (GM == 4 || GM == 8);  // tensor-core chunks (16-slot ones)
+    const bool mm_ok = q4 && c.dtype == KVC_BF16;  // tensor-core chunks (16-slot ones)
     if (aligned && (two || mm_ok)) {
-        const int RL = GM / 2, cap_w = (256 / (RL + 1)) / 8 * 8;  // the kernel's RL and kTmCap
+        const int RL = GM <= 2 ? 1 : GM / 2, cap_w = (256 / (RL + 1)) / 8 * 8;  // the kernel's RL and kTmCap
         for (int CH = std::min(16, c.page_size); CH >= 4; --CH) {
             if (c.page_size % CH || CH % 4 || c.max_slots % CH) continue;
             const bool mm = mm_ok && CH == 16;
@@ -1029,7 +1065,7 @@ cudaError_t launch_t(const CacheView &c, const void *q, const int32_t *q_pos, in
 template <typename T, int D, int GM>
 cudaError_t launch_r(const CacheView &c, const void *q, const int32_t *q_pos, int32_t num_q_heads, float *out,
                      float *lse, float *scores, bool accumulate, int32_t *status, cudaStream_t stream, const Plan &p) {
-    if constexpr ((GM == 4 || GM == 8) && sizeof(T) == 2) {
+    if constexpr (sizeof(T) == 2) {
         if (p.mm)
             return launch_t<T, D, GM, kTmRing, true, true>(c, q, q_pos, num_q_heads, out, lse, scores, accumulate,
                                                            status, stream, p);

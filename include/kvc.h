@@ -405,14 +405,15 @@ kvc_status kvc_beacon_update(const void *q, const int32_t *num_q, int32_t num_se
  * Limits:  num_q_heads / num_kv_heads <= 8.  Each CTA of the row's cluster (at most 8 CTAs) keeps
  *          its slice's logits until the row's LSE is known, in one of two places (G' = the group
  *          size rounded up to a power of two):
- *          - tensor memory, when slot_pos and scores start on 16-byte boundaries, G' is 2 or 4 at
- *            head_dim 128 (2, 4 or 8 at head_dim 64), or G' is 8 with bf16, 16-slot chunks and a
- *            4-byte aligned q, and the page size has a divisor that is a multiple of 4: the stages
- *            then also carry the chunk's positions and old scores, and every warp keeps two chunks
- *            in flight.  Rows up to 131,072 / 81,920 / 49,152 slots at G' = 2 / 4 / 8 with 16-slot
- *            chunks.  With bf16, G' = 4 or 8 and a 4-byte aligned q, each chunk's q . k and
- *            probability-weighted V sums run on the tensor cores (fp32 accumulation; the
- *            probabilities enter as a bf16 pair that keeps 16 bits of mantissa);
+ *          - tensor memory, when slot_pos and scores start on 16-byte boundaries, the page size
+ *            has a divisor that is a multiple of 4, and either the cache is bf16 with 16-slot
+ *            chunks and a 4-byte aligned q (any G'), or G' is 2 or 4 at head_dim 128 (2, 4 or 8
+ *            at head_dim 64): the stages then also carry the chunk's positions and old scores,
+ *            and every warp keeps two chunks in flight.  Rows up to 131,072 / 81,920 / 49,152
+ *            slots at G' <= 2 / 4 / 8 with 16-slot chunks.  With bf16, 16-slot chunks and a
+ *            4-byte aligned q, each chunk's q . k and probability-weighted V sums run on the
+ *            tensor cores (fp32 accumulation; the probabilities enter as a bf16 pair that keeps
+ *            16 bits of mantissa);
  *          - otherwise shared memory: (G' + 1) * 4 * ceil(max_slots / 8) bytes of logits and
  *            positions beside at least two K/V stages per warp, within 218 KiB; a stage holds a
  *            chunk of 16 slots of one page, shrinking to 8, 4, 2 or 1 slots (slower) when 16 do

@@ -100,6 +100,10 @@ CASES = {
     # 8-token pages: 8-slot chunks, so the dot products run on the FMA pipes with the logits in TMEM (G = 4)
     # and in shared memory (G = 8)
     "pages8_gqa4": dict(ctx=(2500, 777), S=2, seed=50, P=8),
+    # one and two query heads per KV head on the tensor-core chunks
+    "mha_bf16": dict(Hq=8, Hkv=8, ctx=(2600,), seed=53),
+    "gqa2_bf16": dict(Hq=16, Hkv=8, ctx=(1500, 2222), S=2, seed=54),
+    "mha_bf16_d64": dict(Hq=4, Hkv=4, D=64, ctx=(3100,), seed=55),
     "pages8_gqa8": dict(Hq=64, Hkv=8, ctx=(1900,), seed=51, P=8),
     # 12-token pages: 12-slot chunks (not a power of two)
     "pages12_gqa4": dict(ctx=(2000,), seed=52, P=12),
